@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one decode step of a batch: for every layer, pa_copy_blocks of
+the copy-on-write pairs (parallel-sampling workload only), pa_reshape_and_cache
+of one new token per sequence, then pa_decode over the whole paged context.
+Inputs are resident in HBM before the timed region; each layer has its own
+KV cache (all larger than the 126 MB L2, so no flush is needed).  Prints one
+JSON line: tokens/s (`value`), the decode call's achieved HBM GB/s against
+the measured copy bandwidth (`roofline`), the same metric through host
+buffers (`e2e`), and the fp64 CPU oracle timed on a bounded sample
+(`cpu_baseline`).
+
+N > 1 (torchrun): every rank runs its own replica of the workload on its
+GPU (sequences are independent, so there is no data-path exchange; weak
+scaling); the time is the max over ranks.
+
+`--impl reference` times the CPU oracle itself on the same workload (rank 0
+only), each step a bounded sample of it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode attention tokens/s and achieved KV GB/s as % of B200 HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b",
+                    choices=["llama7b", "llama13b", "gqa_long", "cow", "tiny"])
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layer caches to allocate (0: the workload's layer count; fewer "
+                         "caches are cycled so every step still runs every layer)")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the CPU-oracle sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- distributed helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over the process group (identity when alone)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- workload description
+def algorithmic_bytes(lens, num_q_heads, num_kv_heads, head_dim, elem=2, block=16) -> int:
+    """Bytes one pa_decode call must move: K and V of every cached token, q and
+    out, the block-table entries it reads and the context lengths."""
+    lens = np.asarray(lens, dtype=np.int64)
+    S = len(lens)
+    kv = int(2 * lens.sum() * num_kv_heads * head_dim * elem)
+    qo = 2 * S * num_q_heads * head_dim * elem
+    tables = int(4 * ((lens + block - 1) // block).sum())
+    return kv + qo + tables + 4 * S
+
+
+def describe(w: wl.Workload, lens, layers_alloc: int) -> dict:
+    return {
+        "workload": w.name,
+        "num_seqs": int(len(lens)),
+        "num_q_heads": w.num_q_heads,
+        "num_kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim,
+        "block_size": w.block_size,
+        "layers_per_step": w.layers,
+        "layer_caches": layers_alloc,
+        "context_lens": f"{w.lens}; mean {float(np.mean(lens)):.1f}, max {int(np.max(lens))}",
+        "l2": "inputs larger than L2: every layer call streams its own KV cache (> 126 MB)",
+        "seed": 0,
+    }
+
+
+def load_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("pa_kernels.cuh", "pa_device.cuh", "pa_api.cu"):
+        with open(os.path.join(ROOT, "paged_kv_cache_425_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_call(workload: str, calls_bytes: int):
+    """ncu DRAM bytes of one decode call, scaled to this call, if the record
+    matches the current kernel sources; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_digest") != kernel_source_digest():
+        return None
+    r = rec.get("workloads", {}).get(workload)
+    if not r:
+        return None
+    return int(r["dram_bytes_per_call"] * calls_bytes / r["algorithmic_bytes_per_call"])
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"pa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == 7 and parts[0].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[3:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][1]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- our arm
+class Setup:
+    """Device-resident inputs of one workload (one replica)."""
+
+    def __init__(self, args, device, rank):
+        import torch
+        import paged_kv_cache_425_b200 as pk
+        from paged_kv_cache_425_b200 import batch
+        self.pk = pk
+        w = wl.WORKLOADS[args.workload]
+        self.w = w
+        rng = wl.rng_for(args.seed + rank)
+        tdt = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+        self.tdt = tdt
+        t0 = time.time()
+        if args.workload == "cow":
+            own = wl.draw_branch_tokens(w, rng)
+            nb = batch.cow_pool_blocks(w)
+            fb = batch.ForkedBatch(w, own, wl.draw_block_order(nb, rng), nb)
+            b = fb.step()  # the divergence step: every branch copies or writes in place
+        else:
+            lens = wl.draw_context_lens(w, rng)
+            nb = wl.pool_size(w, lens)
+            b = batch.decode_batch(w, lens, wl.draw_block_order(nb, rng), nb,
+                                   batch.max_blocks_for(w))
+        self.alloc_seconds = time.time() - t0
+        self.batch = b
+        self.S = len(b.seq_ids)
+        self.nb = nb
+        self.layers = w.layers
+        self.ncache = args.layers if args.layers > 0 else w.layers
+        self.ncache = min(self.ncache, w.layers)
+        H, Hq, d = w.num_kv_heads, w.num_q_heads, w.head_dim
+        gen = torch.Generator(device=device)
+        gen.manual_seed(1000 + args.seed + rank)
+        shape = (nb, H, 16, d)
+        self.kc = [torch.randn(shape, generator=gen, device=device, dtype=tdt)
+                   for _ in range(self.ncache)]
+        self.vc = [torch.randn(shape, generator=gen, device=device, dtype=tdt)
+                   for _ in range(self.ncache)]
+        L = self.layers
+        self.q = torch.randn((L, self.S, Hq, d), generator=gen, device=device, dtype=tdt)
+        self.k_new = torch.randn((L, self.S, H, d), generator=gen, device=device, dtype=tdt)
+        self.v_new = torch.randn((L, self.S, H, d), generator=gen, device=device, dtype=tdt)
+        self.out = torch.empty((L, self.S, Hq, d), device=device, dtype=tdt)
+        self.tables = torch.from_numpy(b.tables).to(device)
+        self.lens = torch.from_numpy(b.context_lens).to(device)
+        self.slots = torch.from_numpy(b.slots).to(device)
+        self.pairs = torch.from_numpy(b.pairs).to(device) if len(b.pairs) else None
+        nws = pk.decode_workspace_size(self.S, Hq, d, b.max_blocks)
+        self.ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=device) if nws else None
+        self.parts = (b.max_blocks + 31) // 32
+        self.stream = torch.cuda.current_stream(device)
+        self.bytes_per_call = algorithmic_bytes(b.context_lens, Hq, H, d)
+        self.launches_per_step = L * (1 + 1 + (1 if self.parts > 1 else 0)
+                                      + (1 if self.pairs is not None else 0))
+
+    def step(self, ev=None):
+        pk, w = self.pk, self.w
+        for l in range(self.layers):
+            c = l % self.ncache
+            if self.pairs is not None:
+                pk.copy_blocks(self.kc[c], self.vc[c], self.pairs, stream=self.stream)
+            pk.reshape_and_cache(self.k_new[l], self.v_new[l], self.kc[c], self.vc[c], self.slots,
+                                 stream=self.stream)
+            if ev is not None:
+                ev[0][l].record(self.stream)
+            pk.decode(self.out[l], self.q[l], self.kc[c], self.vc[c], self.tables, self.lens,
+                      w.num_kv_heads, w.scale, workspace=self.ws, stream=self.stream)
+            if ev is not None:
+                ev[1][l].record(self.stream)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    st = Setup(args, device, rank)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        st.step()
+    rc, bits = st.pk.get_error(st.stream)
+    if rc != 0:
+        raise RuntimeError(f"device error word {bits:#x} during warm-up")
+
+    # ---- device-resident timing
+    L = st.layers
+    dec_ms = []
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    barrier(device)
+    torch.cuda.synchronize()
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(st.stream)
+    all_ev = []
+    for _ in range(args.steps):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(L)] for _ in range(2)]
+        st.step(ev)
+        all_ev.append(ev)
+    t1.record(st.stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    clocks = sampler.stop()
+    local_ms = t0.elapsed_time(t1)
+    for ev in all_ev:
+        dec_ms += [a.elapsed_time(b) for a, b in zip(ev[0], ev[1])]
+    rc, bits = st.pk.get_error(st.stream)
+    if rc != 0:
+        raise RuntimeError(f"device error word {bits:#x} in the timed region")
+    total_ms = max_over_ranks(local_ms, device)
+    dec_avg_ms = max_over_ranks(float(np.mean(dec_ms)), device)
+
+    # ---- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(st, args, device, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args, st)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak, peak_src = load_peak()
+    achieved = st.bytes_per_call / (dec_avg_ms * 1e-3) / 1e9
+    value = world * st.S * args.steps / (total_ms * 1e-3)
+    traffic = traffic_per_call(args.workload, st.bytes_per_call)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16" if st.w.dtype == wl.F16 else "bf16",
+        "data": "synthetic: seeded N(0,1) q/k/v/cache, seeded context lengths, allocator-built scattered tables",
+        "config": {**describe(st.w, st.batch.context_lens, st.ncache), "parallelism": f"replicas x{world}",
+                   "num_blocks": st.nb, "decode_partitions": st.parts,
+                   "cow_pairs_per_layer": 0 if st.pairs is None else int(st.pairs.shape[0]),
+                   "host_alloc_seconds": round(st.alloc_seconds, 3)},
+        "kv_gbs": round(achieved, 1),
+        "hbm_frac": round(achieved / peak, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "pa_decode call (partition kernel + merge kernel)",
+                     "algorithmic_bytes_per_call": st.bytes_per_call,
+                     "avg_call_us": round(dec_avg_ms * 1e3, 2), "peak_source": peak_src},
+        "gpu_launches": st.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(st, args, device, world):
+    """Same steps, with every step's inputs copied from pinned host memory and
+    its outputs read back, inside the timed region."""
+    import torch
+    hq = st.q.cpu().pin_memory()
+    hk = st.k_new.cpu().pin_memory()
+    hv = st.v_new.cpu().pin_memory()
+    ht = st.tables.cpu().pin_memory()
+    hl = st.lens.cpu().pin_memory()
+    hs = st.slots.cpu().pin_memory()
+    hp = st.pairs.cpu().pin_memory() if st.pairs is not None else None
+    hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    ins = [(st.q, hq), (st.k_new, hk), (st.v_new, hv), (st.tables, ht), (st.lens, hl),
+           (st.slots, hs)] + ([(st.pairs, hp)] if hp is not None else [])
+    h2d = sum(h.numel() * h.element_size() for _, h in ins)
+    d2h = hout.numel() * hout.element_size()
+
+    def one():
+        for dev, host in ins:
+            dev.copy_(host, non_blocking=True)
+        st.step()
+        hout.copy_(st.out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    barrier(device)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(st.stream)
+    for _ in range(args.steps):
+        one()
+    b.record(st.stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    ms = max_over_ranks(a.elapsed_time(b), device)
+    return {"value": round(world * st.S * args.steps / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms / args.steps, 4)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """The fp64 oracle on one layer of the workload, host-generated inputs,
+    over the first sequences of the batch (a bounded sample)."""
+
+    def __init__(self, w: wl.Workload, seed: int, budget_tokens: int):
+        import oracle
+        from paged_kv_cache_425_b200 import batch as pbatch
+        self.oracle = oracle
+        rng = wl.rng_for(seed)
+        if w.name == "cow":
+            own = wl.draw_branch_tokens(w, rng)
+            nb = pbatch.cow_pool_blocks(w)
+            b = pbatch.ForkedBatch(w, own, wl.draw_block_order(nb, rng), nb).step()
+        else:
+            lens = wl.draw_context_lens(w, rng)
+            nb = wl.pool_size(w, lens)
+            b = pbatch.decode_batch(w, lens, wl.draw_block_order(nb, rng), nb,
+                                    pbatch.max_blocks_for(w))
+        lens = b.context_lens
+        n = int(np.searchsorted(np.cumsum(lens), budget_tokens)) + 1
+        self.seqs = np.arange(min(n, len(lens)), dtype=np.int32)
+        self.sample_tokens = int(lens[self.seqs].sum())
+        # only the blocks the sampled sequences use are generated; others stay zero
+        self.w = w
+        self.b = b
+        self.q = wl.draw_values(rng, (len(lens), w.num_q_heads, w.head_dim), w.dtype)
+        used = np.unique(b.tables[self.seqs][b.tables[self.seqs] >= 0])
+        self.kc = np.zeros((nb, w.num_kv_heads, 16, w.head_dim), np.uint16)
+        self.vc = np.zeros_like(self.kc)
+        self.kc[used] = wl.draw_values(rng, (len(used), w.num_kv_heads, 16, w.head_dim), w.dtype)
+        self.vc[used] = wl.draw_values(rng, (len(used), w.num_kv_heads, 16, w.head_dim), w.dtype)
+
+    def run_layer(self):
+        self.oracle.decode(self.q, self.kc, self.vc, self.b.tables, self.b.context_lens,
+                           self.w.num_kv_heads, self.w.scale, self.w.dtype, seqs=self.seqs)
+
+    def describe(self, calls):
+        return (f"{calls} oracle calls of one layer over the first {len(self.seqs)} of "
+                f"{len(self.b.context_lens)} sequences ({self.sample_tokens} cached tokens x "
+                f"{self.w.num_q_heads} q heads); a step = {self.w.layers} such layer calls")
+
+
+def cpu_baseline(args, st):
+    import oracle
+    s = OracleSample(st.w, args.seed, budget_tokens=20000)
+    s.run_layer()  # warm
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        s.run_layer()
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= args.cpu_seconds:
+            break
+    per_layer = el / calls
+    tok_s = len(s.seqs) / (per_layer * st.w.layers)
+    return {"value": round(tok_s, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": s.describe(calls)}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    w = wl.WORKLOADS[args.workload]
+    s = OracleSample(w, args.seed, budget_tokens=4000)
+    for _ in range(args.warmup):
+        s.run_layer()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.run_layer()
+    el = time.perf_counter() - t0
+    per_layer = el / args.steps
+    tok_s = len(s.seqs) / (per_layer * w.layers)
+    ms_step = per_layer * w.layers * 1e3
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(tok_s, 3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: seeded N(0,1) values, seeded context lengths, allocator-built tables",
+        "config": describe(w, s.b.context_lens, 1),
+        "cpu_baseline": {"value": round(tok_s, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": s.describe(args.steps) + "; per-step time = layers x per-call"},
+        "e2e": {"value": round(tok_s, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if world > 1 and args.gpus != world:
+        args.gpus = world
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return 0
+    run_ours(args, world, rank, local)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

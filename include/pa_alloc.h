@@ -1,0 +1,130 @@
+/*
+ * pa_alloc.h - host-side block allocator for the paged KV cache (libpa.so).
+ *
+ * Sources:
+ *  - "Inside vLLM: How PagedAttention Changes Python LLM Inference at the
+ *    Systems Level", section "PagedAttention: What the OS Figured Out Decades
+ *    Ago": the pool is cut into fixed-size blocks; each sequence has a block
+ *    table from logical block index to physical block; blocks are claimed as
+ *    generation proceeds and released as soon as a sequence finishes.
+ *  - same page, section "Copy-on-Write Makes Beam Search Cheap": branches of
+ *    one prompt share its blocks by reference count; only a branch that
+ *    writes into a shared block gets a copy of that block, the rest stays
+ *    shared.
+ *  - same page, section "Python LLM Inference Optimization with vLLM:
+ *    Parameters That Actually Matter": the block pool takes a fraction
+ *    (gpu_memory_utilization) of the memory left after the weights.
+ *  - "vLLM PagedAttention: reducing KV cache memory waste", section "How
+ *    PagedAttention Works": only a sequence's last block can be partly
+ *    empty, so waste is bounded by one block per sequence.
+ *  - same page, section "Why KV Cache Dominates GPU Memory", and "Inside
+ *    vLLM ...", section "The Real Reason Your GPU Memory Is Full When It
+ *    Isn't": KV bytes = 2 x layers x tokens x hidden x bytes per element.
+ *
+ * The allocator is plain host C++ (no CUDA call).  It is not thread-safe:
+ * one thread drives one allocator.  Free blocks are handed out first in,
+ * first out: a freshly created pool hands out 0, 1, 2, ...; a block freed
+ * later goes to the back of the queue.  Every call that fails leaves the
+ * allocator unchanged.
+ */
+#ifndef PA_ALLOC_H
+#define PA_ALLOC_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pa_alloc pa_alloc;
+
+typedef struct {
+    int64_t num_blocks;     /* pool size */
+    int64_t free_blocks;    /* on the free list */
+    int64_t used_blocks;    /* refcount > 0 */
+    int64_t shared_blocks;  /* refcount > 1 */
+    int64_t num_seqs;       /* live sequences */
+    int64_t logical_tokens; /* sum of the sequences' token counts */
+    int64_t logical_blocks; /* sum of the sequences' table lengths */
+    int64_t filled_slots;   /* slots of used blocks that hold a token */
+    int64_t cow_copies;     /* copy pairs emitted since creation */
+    double usage;           /* used_blocks / num_blocks */
+    double waste;           /* 1 - filled_slots / (used_blocks * block_size) */
+    double sharing_saving;  /* 1 - used_blocks / logical_blocks */
+} pa_alloc_stats;
+
+/* New pool of num_blocks blocks of block_size tokens, all free.  NULL on a
+ * non-positive size or out of host memory. */
+pa_alloc *pa_alloc_create(int32_t num_blocks, int32_t block_size);
+void pa_alloc_destroy(pa_alloc *a);
+
+/* Register sequence seq_id holding num_tokens tokens (a prompt) and claim
+ * ceil(num_tokens / block_size) blocks for it.  PA_ERR_INVALID_ARG if the id
+ * exists or num_tokens < 0; PA_ERR_NO_BLOCKS (nothing claimed) if the free
+ * list is too short. */
+int pa_alloc_add_seq(pa_alloc *a, int64_t seq_id, int32_t num_tokens);
+
+/* child_id becomes a branch of parent_id: same tokens, same physical blocks,
+ * every block's refcount + 1.  No block is claimed. */
+int pa_alloc_fork(pa_alloc *a, int64_t parent_id, int64_t child_id);
+
+/* Make room for one more token of seq_id at position p = its token count.
+ * If p starts a new block, claim one and append it to the table.  Else, if
+ * the last block is shared (refcount > 1), claim a fresh block, drop one
+ * reference to the shared one, put the fresh one in the table and report
+ * (*cow_src, *cow_dst) = (shared, fresh): the caller must copy that block
+ * (pa_copy_blocks) before writing the token.  Otherwise the token goes into
+ * the last block in place.  *cow_src = *cow_dst = -1 when no copy is needed.
+ * *slot = table[p / block_size] * block_size + p % block_size.  The token
+ * count becomes p + 1. */
+int pa_alloc_append_slot(pa_alloc *a, int64_t seq_id, int64_t *slot, int32_t *cow_src,
+                         int32_t *cow_dst);
+
+/* pa_alloc_append_slot for n sequences in order.  slots[i] receives the
+ * slot of seq_ids[i]; copy pairs are appended to pairs ([n][2] capacity) and
+ * counted in *num_pairs.  On PA_ERR_NO_BLOCKS the sequences before the
+ * failing one keep their new slot; *num_pairs counts their pairs. */
+int pa_alloc_append_slots(pa_alloc *a, const int64_t *seq_ids, int32_t n, int64_t *slots,
+                          int32_t *pairs, int32_t *num_pairs);
+
+/* Drop seq_id: every block's refcount - 1; blocks reaching 0 go to the back
+ * of the free list at once. */
+int pa_alloc_free_seq(pa_alloc *a, int64_t seq_id);
+
+/* Token count of seq_id, or PA_ERR_INVALID_ARG if unknown. */
+int32_t pa_alloc_num_tokens(const pa_alloc *a, int64_t seq_id);
+
+/* Copy seq_id's block table into out (at most cap entries); returns its
+ * length, or PA_ERR_INVALID_ARG. */
+int32_t pa_alloc_block_table(const pa_alloc *a, int64_t seq_id, int32_t *out, int32_t cap);
+
+/* Padded table matrix for a batch: row i of tables ([n][max_blocks], host)
+ * receives seq_ids[i]'s table followed by -1s; context_lens[i] its token
+ * count.  PA_ERR_INVALID_ARG if a table is longer than max_blocks. */
+int pa_alloc_build_tables(const pa_alloc *a, const int64_t *seq_ids, int32_t n, int32_t *tables,
+                          int32_t max_blocks, int32_t *context_lens);
+
+/* Current reference count of a physical block (0 = free), or -1. */
+int32_t pa_alloc_refcount(const pa_alloc *a, int32_t block);
+
+int pa_alloc_get_stats(const pa_alloc *a, pa_alloc_stats *out);
+
+/* KV bytes one token occupies across all layers: 2 x layers x kv_heads x
+ * head_dim x dtype_bytes (K and V). */
+int64_t pa_kv_bytes_per_token(int32_t layers, int32_t kv_heads, int32_t head_dim,
+                              int32_t dtype_bytes);
+
+/* Pool bytes for a GPU: utilization x (gpu_bytes - weight_bytes), 0 if the
+ * weights do not fit. */
+double pa_pool_bytes(double gpu_bytes, double weight_bytes, double utilization);
+
+/* Blocks that fit in pool_bytes for a model of that shape:
+ * floor(pool_bytes / (block_size x pa_kv_bytes_per_token(...))). */
+int64_t pa_pool_num_blocks(double pool_bytes, int32_t layers, int32_t kv_heads, int32_t head_dim,
+                           int32_t block_size, int32_t dtype_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_ALLOC_H */

@@ -1,0 +1,195 @@
+/*
+ * pa_api.h - C ABI of the paged KV-cache decode library (libpa.so).
+ *
+ * The library implements the data-parallel hot path of PagedAttention on
+ * NVIDIA B200 (sm_100a): writing each new token's K/V into its slot of a
+ * block-paged cache, copying shared blocks on write, and single-token decode
+ * attention that reaches every cached token through a per-sequence block
+ * table.
+ *
+ * Sources of the operations (web pages on PagedAttention):
+ *  - "Inside vLLM: How PagedAttention Changes Python LLM Inference at the
+ *    Systems Level", section "PagedAttention: What the OS Figured Out
+ *    Decades Ago": fixed-size blocks of 16 tokens, a block table mapping
+ *    logical to physical blocks, non-contiguous blocks that attention sees as
+ *    contiguous, new blocks appended as tokens are generated.
+ *  - same page, section "Copy-on-Write Makes Beam Search Cheap": shared
+ *    prefix blocks by reference count; a write into a shared block copies
+ *    that block only.
+ *  - "vLLM PagedAttention: reducing KV cache memory waste", section "How
+ *    PagedAttention Works": blocks claimed on demand, waste only in the last
+ *    block, copy-on-write on divergence.
+ *  - "PagedAttention in vLLM: a throughput settings guide", section
+ *    "Continuous Batching Keeps the GPU Busy": decoding is bound by memory
+ *    bandwidth.
+ *
+ * Conventions shared by every call:
+ *  - Pointers marked "device" are CUDA device addresses on the current
+ *    device; "host" pointers are ordinary host memory.  The caller owns every
+ *    buffer.  The library allocates no device memory: scratch (workspace) is
+ *    passed in by the caller.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    except pa_get_error only enqueues work on `stream` and returns.
+ *  - Element types: PA_F16 (IEEE binary16) or PA_BF16 (bfloat16), 2 bytes.
+ *  - Cache layout: key_cache and value_cache are each
+ *      [num_blocks][num_kv_heads][block_size][head_dim]
+ *    with head_dim contiguous, so one (block, kv head) tile of block_size
+ *    rows is contiguous (4 KiB at head_dim 128).  Element (b, h, o, i) is at
+ *    ((b * num_kv_heads + h) * block_size + o) * head_dim + i.
+ *    Both caches must start on a 16-byte boundary.
+ *  - Supported shapes: block_size == 16 (PA_BLOCK_SIZE), head_dim 64 or 128,
+ *    num_q_heads a multiple of num_kv_heads with at most 16 query heads per
+ *    kv head, num_blocks * num_kv_heads * 16 < 2^31.  Anything else returns
+ *    PA_ERR_UNSUPPORTED (or PA_ERR_INVALID_ARG for inconsistent values)
+ *    before any work is enqueued.
+ *  - Bad indices found on the device (a block id outside [0, num_blocks), a
+ *    slot outside the pool, a context length above the table's capacity) are
+ *    never dereferenced: the kernel skips the access and sets a bit in the
+ *    library's device error word, which pa_get_error reads and clears.
+ *  - Return value: PA_OK or a negative pa_status.  A launch failure reported
+ *    by the CUDA runtime returns PA_ERR_CUDA.
+ */
+#ifndef PA_API_H
+#define PA_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = -1,  /* null pointer, negative size, inconsistent shapes */
+    PA_ERR_UNSUPPORTED = -2,  /* valid but not built: block_size, head_dim, dtype, group */
+    PA_ERR_OUT_OF_RANGE = -3, /* pa_get_error: the device saw a bad index */
+    PA_ERR_NO_BLOCKS = -4,    /* allocator: the free list cannot serve the request */
+    PA_ERR_CUDA = -5,         /* the CUDA runtime reported an error */
+    PA_ERR_WORKSPACE = -6,    /* pa_decode: workspace missing or too small */
+    PA_ERR_TIMEOUT = -7       /* pa_get_error: a device wait gave up */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+#define PA_BLOCK_SIZE 16
+/* Decode splits a context into partitions of this many tokens (32 blocks). */
+#define PA_PARTITION_TOKENS 512
+
+/* Bits of the device error word (pa_get_error). */
+#define PA_DEVERR_BLOCK_ID 1u    /* block table entry outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 2u        /* slot_mapping entry >= num_blocks * block_size */
+#define PA_DEVERR_PAIR 4u        /* copy pair id outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 8u /* context_len < 0 or > max_blocks_per_seq * block_size */
+#define PA_DEVERR_TIMEOUT 16u    /* a bounded wait on an async copy gave up */
+
+/*
+ * pa_reshape_and_cache - write the new tokens' K and V into their cache slots.
+ *
+ * Source: "Inside vLLM ...", section "PagedAttention: What the OS Figured Out
+ * Decades Ago" (a sequence's tokens live in the blocks its table lists; new
+ * tokens go into the table's last block, or a newly appended one).
+ *
+ * For each token t with slot = slot_mapping[t] >= 0:
+ *   key_cache  [slot / block_size][h][slot % block_size][:] = k[t][h][:]
+ *   value_cache[slot / block_size][h][slot % block_size][:] = v[t][h][:]
+ * for every kv head h.  The slot of a token at position p of a sequence is
+ * table[p / block_size] * block_size + p % block_size (pa_alloc_append_slot
+ * returns it).  A negative slot is padding and is skipped.  A slot at or
+ * beyond num_blocks * block_size is skipped and sets PA_DEVERR_SLOT.
+ * The copy is bit-exact.  Two tokens with the same slot race (undefined
+ * which one lands).
+ *
+ *   k, v          device, [num_tokens][num_kv_heads][head_dim], dtype,
+ *                 contiguous, 16-byte aligned
+ *   key_cache,    device, cache layout above (written in place)
+ *   value_cache
+ *   slot_mapping  device, int64 [num_tokens]
+ */
+int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *value_cache,
+                         const int64_t *slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, int64_t num_blocks, int32_t dtype,
+                         void *stream);
+
+/*
+ * pa_decode - single-token decode attention over the paged cache.
+ *
+ * Source: "Inside vLLM ...", section "PagedAttention: What the OS Figured Out
+ * Decades Ago" (the block table makes scattered blocks look contiguous to
+ * attention); "PagedAttention in vLLM: a throughput settings guide", section
+ * "Continuous Batching Keeps the GPU Busy" (decode reads memory, not math).
+ *
+ * For sequence s with L = context_lens[s] cached tokens (the new token
+ * included, written beforehand by pa_reshape_and_cache) and query head h,
+ * with G = num_q_heads / num_kv_heads and kv head g = h / G:
+ *   K_j = key_cache  [block_tables[s][j / 16]][g][j % 16][:],  j < L
+ *   V_j = value_cache[block_tables[s][j / 16]][g][j % 16][:]
+ *   out[s][h][:] = sum_j softmax_j(scale * q[s][h] . K_j) V_j
+ * Products and the softmax are computed in fp32; out is rounded to dtype.
+ * L == 0 gives a zero row.  Table entries past ceil(L / 16) are not read.
+ *
+ * Contexts longer than PA_PARTITION_TOKENS are split into partitions that
+ * run in parallel and are merged by log-sum-exp; the partial results go to
+ * `workspace`, which must hold pa_decode_workspace_size(...) bytes (256-byte
+ * aligned) whenever max_blocks_per_seq * 16 > PA_PARTITION_TOKENS, and may be
+ * NULL otherwise.  Calls that share a workspace must not overlap.
+ *
+ *   out           device, [num_seqs][num_q_heads][head_dim], dtype
+ *   q             device, [num_seqs][num_q_heads][head_dim], dtype
+ *   key_cache,    device, cache layout above (read only)
+ *   value_cache
+ *   block_tables  device, int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens  device, int32 [num_seqs]
+ *   scale         multiplier of q . k (typically 1 / sqrt(head_dim))
+ */
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *context_lens, int32_t num_kv_heads,
+              float scale, int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace pa_decode needs for these sizes (0 when no context can
+ * exceed one partition). */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_blocks_per_seq);
+
+/*
+ * pa_copy_blocks - copy-on-write block copies.
+ *
+ * Source: "Inside vLLM ...", section "Copy-on-Write Makes Beam Search Cheap";
+ * "vLLM PagedAttention: reducing KV cache memory waste", section "How
+ * PagedAttention Works" (copy-on-write handles divergence of shared blocks).
+ *
+ * For each pair p: physical block src_dst_pairs[p][1] (every kv head, every
+ * row, K and V) becomes a bit-exact copy of block src_dst_pairs[p][0].
+ * Destinations must be distinct and no destination may also be a source in
+ * the same call (pa_alloc_append_slot never produces such pairs); otherwise
+ * the result is undefined.  A pair with an id outside [0, num_blocks) is
+ * skipped and sets PA_DEVERR_PAIR.
+ *
+ *   src_dst_pairs  device, int32 [num_pairs][2]
+ */
+int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pairs,
+                   int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                   int64_t num_blocks, int32_t dtype, void *stream);
+
+/*
+ * pa_get_error - synchronise `stream`, then read and clear the device error
+ * word (one word for the whole process and device).  *bits (host, may be
+ * NULL) receives the PA_DEVERR_* bits seen since the last call.  Returns
+ * PA_OK if no bit was set, PA_ERR_TIMEOUT if PA_DEVERR_TIMEOUT was set,
+ * PA_ERR_OUT_OF_RANGE for any other bit, PA_ERR_CUDA if the stream failed.
+ */
+int pa_get_error(void *stream, uint32_t *bits);
+
+/* Static description of a status code. */
+const char *pa_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_API_H */

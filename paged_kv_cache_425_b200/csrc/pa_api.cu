@@ -1,0 +1,270 @@
+// Host side of libpa.so: argument checks, TMA descriptor encoding and kernel
+// launches for the entry points declared in include/pa_api.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pa_api.h"
+#include "pa_kernels.cuh"
+
+namespace pa {
+namespace {
+
+// Decode launch shape: warps per CTA and TMA stages per warp.
+constexpr int kWarps = 4;
+constexpr int kStages128 = 3;  // 3 x 8 KiB per warp at head_dim 128
+constexpr int kStages64 = 4;   // 4 x 4 KiB per warp at head_dim 64
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// TMA descriptor of a cache viewed as 2-D: rows = num_blocks * num_kv_heads *
+// 16 (one per token slot), columns = head_dim; box = 16 rows x 64 columns
+// (128 bytes), 128-byte swizzle.
+bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int num_kv_heads,
+                      int head_dim, int dtype) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)head_dim,
+                          (cuuint64_t)num_blocks * (cuuint64_t)num_kv_heads * kBlock};
+    cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kBlock};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    2, const_cast<void *>(cache), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_cache_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                      int64_t num_blocks, int32_t dtype) {
+    if (num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+    if (block_size != kBlock) return PA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (num_blocks * (int64_t)num_kv_heads * kBlock >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+template <typename Kernel>
+bool set_smem(Kernel k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+           cudaSuccess;
+}
+
+template <typename T, int D>
+int launch_decode(const DecodeArgs &a, int group, const CUtensorMap &tmk, const CUtensorMap &tmv,
+                  cudaStream_t st) {
+    constexpr int STAGES = D == 128 ? kStages128 : kStages64;
+    constexpr int SMEM = kWarps * STAGES * WarpPipe<D, STAGES>::kStage + 1024;
+    dim3 grid(a.num_parts, a.num_kv_heads, a.num_seqs);
+    dim3 block(kWarps * 32);
+    if (group == 1) {
+        auto k = decode_simt_kernel<T, D, kWarps, STAGES>;
+        if (!set_smem(k, SMEM)) return PA_ERR_CUDA;
+        k<<<grid, block, SMEM, st>>>(tmk, tmv, a);
+    } else if (group <= 8) {
+        auto k = decode_mma_kernel<T, D, kWarps, STAGES, 1>;
+        if (!set_smem(k, SMEM)) return PA_ERR_CUDA;
+        k<<<grid, block, SMEM, st>>>(tmk, tmv, a);
+    } else {
+        auto k = decode_mma_kernel<T, D, kWarps, STAGES, 2>;
+        if (!set_smem(k, SMEM)) return PA_ERR_CUDA;
+        k<<<grid, block, SMEM, st>>>(tmk, tmv, a);
+    }
+    int rc = launch_status();
+    if (rc != PA_OK || a.num_parts <= 1) return rc;
+    merge_kernel<T, D><<<a.num_seqs * a.num_q_heads, kMergeThreads,
+                         a.num_parts * sizeof(float), st>>>(a);
+    return launch_status();
+}
+
+template <typename T>
+int dispatch_decode(const DecodeArgs &a, int head_dim, int group, const CUtensorMap &tmk,
+                    const CUtensorMap &tmv, cudaStream_t st) {
+    return head_dim == 128 ? launch_decode<T, 128>(a, group, tmk, tmv, st)
+                           : launch_decode<T, 64>(a, group, tmk, tmv, st);
+}
+
+int64_t num_parts_for(int32_t max_blocks_per_seq) {
+    return (max_blocks_per_seq + kPartBlocks - 1) / kPartBlocks;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *value_cache,
+                         const int64_t *slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, int64_t num_blocks, int32_t dtype,
+                         void *stream) {
+    int rc = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(key_cache, 16) ||
+        !aligned(value_cache, 16) || !aligned(slot_mapping, 8))
+        return PA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long num_slots = num_blocks * kBlock;
+    const int threads = 256;
+    if (head_dim == 128)
+        scatter_kernel<128><<<num_tokens, threads, 0, st>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+            static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), slot_mapping,
+            num_kv_heads, num_slots);
+    else
+        scatter_kernel<64><<<num_tokens, threads, 0, st>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+            static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), slot_mapping,
+            num_kv_heads, num_slots);
+    return launch_status();
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_blocks_per_seq) {
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || block_size != kBlock ||
+        max_blocks_per_seq <= 0)
+        return 0;
+    const int64_t parts = num_parts_for(max_blocks_per_seq);
+    if (parts <= 1) return 0;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
+    // partition outputs, then (max, sum) pairs, each 256-byte aligned
+    const int64_t o_bytes = (rows * head_dim * 4 + 255) / 256 * 256;
+    const int64_t ml_bytes = (rows * 8 + 255) / 256 * 256;
+    return (size_t)(o_bytes + ml_bytes);
+}
+
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *context_lens, int32_t num_kv_heads,
+              float scale, int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
+              void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    const int group = num_q_heads / num_kv_heads;
+    if (group > 16) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || !aligned(q, 8) ||
+        !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return PA_ERR_INVALID_ARG;
+    const int64_t parts = num_parts_for(max_blocks_per_seq);
+    if (parts > 8192) return PA_ERR_UNSUPPORTED;
+
+    DecodeArgs a;
+    a.out = out;
+    a.q = q;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.ws_o = nullptr;
+    a.ws_ml = nullptr;
+    a.num_blocks = num_blocks;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_parts = (int)parts;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    if (parts > 1) {
+        const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, block_size,
+                                                     max_blocks_per_seq);
+        if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+            return PA_ERR_WORKSPACE;
+        const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
+        const int64_t o_bytes = (rows * head_dim * 4 + 255) / 256 * 256;
+        a.ws_o = static_cast<float *>(workspace);
+        a.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + o_bytes);
+    }
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
+        !encode_cache_map(&tmv, value_cache, num_blocks, num_kv_heads, head_dim, dtype))
+        return PA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return dtype == PA_F16 ? dispatch_decode<__half>(a, head_dim, group, tmk, tmv, st)
+                           : dispatch_decode<__nv_bfloat16>(a, head_dim, group, tmk, tmv, st);
+}
+
+int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pairs,
+                   int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                   int64_t num_blocks, int32_t dtype, void *stream) {
+    int rc = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (rc != PA_OK) return rc;
+    if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!key_cache || !value_cache || !src_dst_pairs) return PA_ERR_INVALID_ARG;
+    if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || !aligned(src_dst_pairs, 4))
+        return PA_ERR_INVALID_ARG;
+    const long long vec_per_block = (long long)num_kv_heads * kBlock * head_dim / 8;
+    const int threads = 256;
+    long long chunks = (vec_per_block + threads * 4 - 1) / (threads * 4);
+    if (chunks > 65535) chunks = 65535;
+    dim3 grid(num_pairs < 65535 ? num_pairs : 65535, (unsigned)chunks);
+    copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), src_dst_pairs,
+        num_pairs, num_blocks, vec_per_block);
+    return launch_status();
+}
+
+int pa_get_error(void *stream, uint32_t *bits) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return PA_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (bits) *bits = word;
+    if (!word) return PA_OK;
+    return (word & PA_DEVERR_TIMEOUT) ? PA_ERR_TIMEOUT : PA_ERR_OUT_OF_RANGE;
+}
+
+const char *pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case PA_ERR_OUT_OF_RANGE: return "device saw an out-of-range index";
+        case PA_ERR_NO_BLOCKS: return "no free blocks";
+        case PA_ERR_CUDA: return "CUDA runtime error";
+        case PA_ERR_WORKSPACE: return "workspace missing or too small";
+        case PA_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int pa_version(void) { return 100; }
+
+}  // extern "C"

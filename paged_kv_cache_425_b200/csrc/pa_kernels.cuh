@@ -1,0 +1,686 @@
+// Kernels of the paged KV-cache hot path for B200 (sm_100a).
+//
+//  * scatter_kernel      - pa_reshape_and_cache: one CTA per new token,
+//                          16-byte vectors, K and V rows to their slot.
+//  * copy_blocks_kernel  - pa_copy_blocks: 16-byte vector copy of whole
+//                          blocks (all kv heads, K and V).
+//  * decode_simt_kernel  - pa_decode with one query head per kv head.
+//  * decode_mma_kernel   - pa_decode with 2..16 query heads per kv head: the
+//                          query group is one mma.sync tile against each
+//                          16-token K / V tile.
+//  * merge_kernel        - log-sum-exp merge of context partitions.
+//
+// Decode grid: (partition, kv head, sequence).  A partition covers
+// PA_PARTITION_TOKENS tokens (32 blocks).  Inside a CTA each warp owns every
+// NW-th block of the partition and runs its own STAGES-deep TMA pipeline:
+// one lane loads the warp's next (block, kv head) K and V tiles with
+// cp.async.bulk.tensor into a 128-byte-swizzled shared-memory stage and an
+// mbarrier tracks the bytes; the warp folds each 16-token tile into a
+// running (max, sum, accumulator) online softmax in fp32, log2 domain.  At
+// the end the CTA combines its warps; a single-partition sequence writes
+// `out`, a split one writes (o, max, sum) to the workspace for merge_kernel.
+//
+// Tile layout in shared memory (matches the TMA 128-byte swizzle): a 16 x D
+// tile is stored as D/64 sub-tiles of 16 rows x 128 bytes; the 16-byte chunk
+// c of row r of a sub-tile sits at chunk position c ^ (r & 7).
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+constexpr int kBlock = 16;                                  // tokens per block
+constexpr int kPartBlocks = PA_PARTITION_TOKENS / kBlock;   // blocks per partition
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;          // 2 s per wait
+
+struct DecodeArgs {
+    void *out;
+    const void *q;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    float *ws_o;    // [S][Hq][P][D]  normalised partition outputs
+    float2 *ws_ml;  // [S][Hq][P]     (max logit in log2 units, sum of 2^(x - max))
+    long long num_blocks;
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int max_blocks_per_seq;
+    int num_parts;     // partitions per sequence in the grid
+    float scale_log2;  // scale * log2(e)
+};
+
+__device__ __forceinline__ int clamp_context(const DecodeArgs &a, int s, bool report) {
+    int L = a.context_lens[s];
+    const int cap = a.max_blocks_per_seq * kBlock;
+    if (L < 0 || L > cap) {
+        if (report) flag_error(PA_DEVERR_CONTEXT_LEN);
+        L = L < 0 ? 0 : cap;
+    }
+    return L;
+}
+
+// Byte offset of 16-byte chunk `chunk` of row r in a swizzled 16 x D tile.
+__device__ __forceinline__ uint32_t tile_off(int r, int chunk) {
+    return (uint32_t)((chunk >> 3) * 2048 + r * 128 + (((chunk & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint8_t *align_smem_1024(uint8_t *p) {
+    const uint32_t base = smem_addr(p);
+    return p + ((1024u - (base & 1023u)) & 1023u);
+}
+
+// Sum-reduce 16 per-lane partial dot products across the warp so that lane
+// l ends up holding the full sum of value (l >> 1): each xor step keeps the
+// half of the values this lane is responsible for and adds the partner's.
+__device__ __forceinline__ float reduce16_scatter(float (&v)[16], int lane) {
+    const unsigned FULL = 0xffffffffu;
+    const bool u4 = lane & 16, u3 = lane & 8, u2 = lane & 4, u1 = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float send = u4 ? v[i] : v[i + 8];
+        const float keep = u4 ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = u3 ? v[i] : v[i + 4];
+        const float keep = u3 ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = u2 ? v[i] : v[i + 2];
+        const float keep = u2 ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 4);
+    }
+    {
+        const float send = u1 ? v[0] : v[1];
+        const float keep = u1 ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(FULL, send, 2);
+    }
+    return v[0] + __shfl_xor_sync(FULL, v[0], 1);
+}
+
+// Per-warp TMA pipeline over the warp's blocks of one partition.
+template <int D, int STAGES>
+struct WarpPipe {
+    static constexpr int kTile = kBlock * D * 2;  // bytes of one K (or V) tile
+    static constexpr int kStage = 2 * kTile;      // K tile then V tile
+
+    uint8_t *ring;
+    uint64_t *bar;
+    const CUtensorMap *tmk;
+    const CUtensorMap *tmv;
+    uint64_t policy;
+    int my_phys;  // lane i: physical block of the warp's i-th block, -1 if none/bad
+    int kvh, num_kv_heads, lane;
+
+    // Issue the loads of the warp's k-th block into stage k % STAGES.
+    // Called by the whole warp; lane 0 issues.
+    __device__ __forceinline__ void issue(int k) {
+        const int phys = __shfl_sync(0xffffffffu, my_phys, k);
+        if (lane == 0) {
+            uint64_t *b = &bar[k % STAGES];
+            uint8_t *dst = ring + (k % STAGES) * kStage;
+            if (phys >= 0) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(b, kStage);
+                const int y = (phys * num_kv_heads + kvh) * kBlock;
+#pragma unroll
+                for (int x = 0; x < D; x += 64) {
+                    tma_load_2d_hint(dst + (x / 64) * 2048, tmk, b, x, y, policy);
+                    tma_load_2d_hint(dst + kTile + (x / 64) * 2048, tmv, b, x, y, policy);
+                }
+            } else {
+                mbar_arrive(b);  // bad id: the stage completes empty
+            }
+        }
+    }
+
+    // Bounded wait for the k-th block; warp-uniform result.
+    __device__ __forceinline__ bool wait(int k) {
+        const bool ok = mbar_wait_bounded(&bar[k % STAGES], (k / STAGES) & 1, kWaitTimeoutNs);
+        return __all_sync(0xffffffffu, ok);
+    }
+
+    // After a failed wait at block k: wait (bounded) for loads still in flight.
+    __device__ __forceinline__ void drain(int k, int issued) {
+        for (int j = k; j < issued; ++j)
+            if (!mbar_wait_bounded(&bar[j % STAGES], (j / STAGES) & 1, kWaitTimeoutNs)) break;
+    }
+};
+
+// Common prologue of both decode kernels.  Returns false if this CTA has no
+// partition to process (it may still have written a zero row).
+struct PartitionInfo {
+    int L, nblk, nparts, b_begin, nk;
+};
+
+__device__ __forceinline__ int warp_block_count(int nb_local, int warp, int nw) {
+    return warp < nb_local ? (nb_local - warp + nw - 1) / nw : 0;
+}
+
+// ------------------------------------------------------------------ decode: one q head per kv head
+template <typename T, int D, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32)
+    decode_simt_kernel(const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a) {
+    using Pipe = WarpPipe<D, STAGES>;
+    constexpr int EPL = D / 32;  // elements of the head dim per lane
+    static_assert(EPL == 2 || EPL == 4, "head_dim 64 or 128");
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[NW][STAGES];
+    __shared__ __align__(16) float s_p[NW][kBlock];
+    __shared__ __align__(16) float s_acc[NW][D];
+    __shared__ float s_m[NW], s_l[NW];
+
+    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int L = clamp_context(a, s, part == 0 && kvh == 0 && threadIdx.x == 0);
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
+    if (part >= (nparts > 0 ? nparts : 1)) return;
+    const size_t row = (size_t)s * a.num_q_heads + kvh;  // q head == kv head
+    uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + row * D;
+    if (nblk == 0) {
+        for (int i = threadIdx.x; i < D; i += NW * 32) out[i] = 0;
+        return;
+    }
+    const int b_begin = part * kPartBlocks;
+    const int nb_local = min(kPartBlocks, nblk - b_begin);
+    const int nk = warp_block_count(nb_local, warp, NW);
+
+    Pipe pipe;
+    pipe.ring = align_smem_1024(dyn_smem) + warp * STAGES * Pipe::kStage;
+    pipe.bar = bars[warp];
+    pipe.tmk = &tmk;
+    pipe.tmv = &tmv;
+    pipe.policy = l2_policy_evict_first();
+    pipe.kvh = kvh;
+    pipe.num_kv_heads = a.num_kv_heads;
+    pipe.lane = lane;
+    pipe.my_phys = -1;
+    if (lane < nk) {
+        const int phys =
+            a.block_tables[(size_t)s * a.max_blocks_per_seq + b_begin + warp + lane * NW];
+        if (phys < 0 || phys >= a.num_blocks)
+            flag_error(PA_DEVERR_BLOCK_ID);
+        else
+            pipe.my_phys = phys;
+    }
+    if (lane == 0) {
+        for (int i = 0; i < STAGES; ++i) mbar_init(&bars[warp][i], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    int issued = nk < STAGES ? nk : STAGES;
+    for (int k = 0; k < issued; ++k) pipe.issue(k);
+
+    float qv[EPL];
+    {
+        const uint16_t *qp = reinterpret_cast<const uint16_t *>(a.q) + row * D + lane * EPL;
+        if constexpr (EPL == 4) {
+            const uint2 raw = *reinterpret_cast<const uint2 *>(qp);
+            const float2 lo = widen2(raw.x, T()), hi = widen2(raw.y, T());
+            qv[0] = lo.x; qv[1] = lo.y; qv[2] = hi.x; qv[3] = hi.y;
+        } else {
+            const float2 f = widen2(*reinterpret_cast<const uint32_t *>(qp), T());
+            qv[0] = f.x; qv[1] = f.y;
+        }
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) qv[i] *= a.scale_log2;
+    }
+
+    float m = -INFINITY, l = 0.f, acc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+    // this lane's 4-byte (EPL 2) or 8-byte (EPL 4) piece of a row: chunk and byte within it
+    const int my_chunk = (lane * EPL) / 8;
+    const int my_byte = ((lane * EPL) % 8) * 2;
+
+    bool dead = false;
+    int k = 0;
+    for (; k < nk; ++k) {
+        if (!pipe.wait(k)) {
+            dead = true;
+            break;
+        }
+        const int phys = __shfl_sync(0xffffffffu, pipe.my_phys, k);
+        const int blk = b_begin + warp + k * NW;
+        const int nvalid = phys >= 0 ? min(kBlock, L - blk * kBlock) : 0;
+        if (nvalid > 0) {
+            const uint8_t *kt = pipe.ring + (k % STAGES) * Pipe::kStage;
+            const uint8_t *vt = kt + Pipe::kTile;
+            float sc[kBlock];
+#pragma unroll
+            for (int t = 0; t < kBlock; ++t) {
+                const uint8_t *src = kt + tile_off(t, my_chunk) + my_byte;
+                if constexpr (EPL == 4) {
+                    const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+                    const float2 lo = widen2(raw.x, T()), hi = widen2(raw.y, T());
+                    sc[t] = qv[0] * lo.x + qv[1] * lo.y + qv[2] * hi.x + qv[3] * hi.y;
+                } else {
+                    const float2 f = widen2(*reinterpret_cast<const uint32_t *>(src), T());
+                    sc[t] = qv[0] * f.x + qv[1] * f.y;
+                }
+            }
+            const int tok = lane >> 1;
+            float x = reduce16_scatter(sc, lane);
+            x = tok < nvalid ? x : -INFINITY;
+            float bm = x;
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const float m_new = fmaxf(m, bm);
+            const float alpha = fast_exp2(m - m_new);
+            const float p = fast_exp2(x - m_new);
+            float ps = p;
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+            l = l * alpha + ps;
+            m = m_new;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) acc[i] *= alpha;
+            if ((lane & 1) == 0) s_p[warp][tok] = p;
+            __syncwarp();
+            float pv[kBlock];
+#pragma unroll
+            for (int i = 0; i < kBlock / 4; ++i) {
+                const float4 f = reinterpret_cast<const float4 *>(s_p[warp])[i];
+                pv[4 * i] = f.x; pv[4 * i + 1] = f.y; pv[4 * i + 2] = f.z; pv[4 * i + 3] = f.w;
+            }
+#pragma unroll
+            for (int t = 0; t < kBlock; ++t) {
+                if (t < nvalid) {
+                    const uint8_t *src = vt + tile_off(t, my_chunk) + my_byte;
+                    if constexpr (EPL == 4) {
+                        const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+                        const float2 lo = widen2(raw.x, T()), hi = widen2(raw.y, T());
+                        acc[0] += pv[t] * lo.x; acc[1] += pv[t] * lo.y;
+                        acc[2] += pv[t] * hi.x; acc[3] += pv[t] * hi.y;
+                    } else {
+                        const float2 f = widen2(*reinterpret_cast<const uint32_t *>(src), T());
+                        acc[0] += pv[t] * f.x; acc[1] += pv[t] * f.y;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (issued < nk) pipe.issue(issued++);
+    }
+    if (dead) {
+        pipe.drain(k, issued);
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) s_acc[warp][lane * EPL + i] = acc[i];
+    if (lane == 0) {
+        s_m[warp] = m;
+        s_l[warp] = l;
+    }
+    __syncthreads();
+
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+        if (s_l[w] > 0.f) M = fmaxf(M, s_m[w]);
+    float wgt[NW], den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        wgt[w] = s_l[w] > 0.f ? fast_exp2(s_m[w] - M) : 0.f;
+        den += wgt[w] * s_l[w];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int i = threadIdx.x; i < D; i += NW * 32) {
+        float o = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            if (wgt[w] != 0.f) o += wgt[w] * s_acc[w][i];
+        o *= inv;
+        if (nparts == 1) {
+            out[i] = narrow1(o, T());
+        } else {
+            a.ws_o[(row * a.num_parts + part) * D + i] = o;
+        }
+    }
+    if (nparts > 1 && threadIdx.x == 0)
+        a.ws_ml[row * a.num_parts + part] = make_float2(den > 0.f ? M : -INFINITY, den);
+}
+
+// ------------------------------------------------------------------ decode: query group on mma.sync
+// NT = number of 8-head column tiles (G <= 8 * NT).
+template <typename T, int D, int NW, int STAGES, int NT>
+__global__ void __launch_bounds__(NW * 32)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const DecodeArgs a) {
+    using Pipe = WarpPipe<D, STAGES>;
+    constexpr int KS = D / 16;     // 16-wide steps of the head dim
+    constexpr int GMAX = 8 * NT;   // query heads per kv head this build handles
+    static_assert(GMAX * D * 4 <= STAGES * Pipe::kStage, "combine scratch fits in a warp ring");
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[NW][STAGES];
+    __shared__ float s_m[NW][GMAX], s_l[NW][GMAX];
+
+    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.num_q_heads / a.num_kv_heads;
+    const int L = clamp_context(a, s, part == 0 && kvh == 0 && threadIdx.x == 0);
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
+    if (part >= (nparts > 0 ? nparts : 1)) return;
+    const size_t row0 = (size_t)s * a.num_q_heads + (size_t)kvh * G;  // first q head of the group
+    uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + row0 * D;
+    if (nblk == 0) {
+        for (int i = threadIdx.x; i < G * D; i += NW * 32) out[i] = 0;
+        return;
+    }
+    const int b_begin = part * kPartBlocks;
+    const int nb_local = min(kPartBlocks, nblk - b_begin);
+    const int nk = warp_block_count(nb_local, warp, NW);
+
+    Pipe pipe;
+    pipe.ring = align_smem_1024(dyn_smem) + warp * STAGES * Pipe::kStage;
+    pipe.bar = bars[warp];
+    pipe.tmk = &tmk;
+    pipe.tmv = &tmv;
+    pipe.policy = l2_policy_evict_first();
+    pipe.kvh = kvh;
+    pipe.num_kv_heads = a.num_kv_heads;
+    pipe.lane = lane;
+    pipe.my_phys = -1;
+    if (lane < nk) {
+        const int phys =
+            a.block_tables[(size_t)s * a.max_blocks_per_seq + b_begin + warp + lane * NW];
+        if (phys < 0 || phys >= a.num_blocks)
+            flag_error(PA_DEVERR_BLOCK_ID);
+        else
+            pipe.my_phys = phys;
+    }
+    if (lane == 0) {
+        for (int i = 0; i < STAGES; ++i) mbar_init(&bars[warp][i], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    int issued = nk < STAGES ? nk : STAGES;
+    for (int k = 0; k < issued; ++k) pipe.issue(k);
+
+    const int g = lane >> 2, c = lane & 3;
+    // B operand of S^T = K Q^T: lane holds Q[h = 8 nt + g][16 kk + 2c .. +1] and [.. + 8 ..].
+    uint32_t qf[NT][KS][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = nt * 8 + g;
+        const uint16_t *qrow = reinterpret_cast<const uint16_t *>(a.q) + (row0 + h) * D;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            qf[nt][kk][0] = h < G ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * c) : 0u;
+            qf[nt][kk][1] =
+                h < G ? *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 8 + 2 * c) : 0u;
+        }
+    }
+    // Running softmax state per (tile nt, head 2c + j), and O^T accumulators:
+    // acc[nt][j] holds rows d = 16 j + g (+8), columns h = 8 nt + 2c (+1).
+    float mrow[NT][2], lrow[NT][2], acc[NT][KS][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        mrow[nt][0] = mrow[nt][1] = -INFINITY;
+        lrow[nt][0] = lrow[nt][1] = 0.f;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) acc[nt][j][0] = acc[nt][j][1] = acc[nt][j][2] = acc[nt][j][3] = 0.f;
+    }
+    // ldmatrix row/chunk of this lane for the K (A, row-major) and V (A^T) tiles
+    const int ka_row = (lane & 7) + ((lane >> 3) & 1) * 8, ka_half = lane >> 4;
+    const int va_row = (lane & 7) + 8 * (lane >> 4), va_half = (lane >> 3) & 1;
+
+    bool dead = false;
+    int k = 0;
+    for (; k < nk; ++k) {
+        if (!pipe.wait(k)) {
+            dead = true;
+            break;
+        }
+        const int phys = __shfl_sync(0xffffffffu, pipe.my_phys, k);
+        const int blk = b_begin + warp + k * NW;
+        const int nvalid = phys >= 0 ? min(kBlock, L - blk * kBlock) : 0;
+        if (nvalid > 0) {
+            uint8_t *kt = pipe.ring + (k % STAGES) * Pipe::kStage;
+            uint8_t *vt = kt + Pipe::kTile;
+            const uint32_t kt_s = smem_addr(kt), vt_s = smem_addr(vt);
+            float sf[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) sf[nt][0] = sf[nt][1] = sf[nt][2] = sf[nt][3] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                uint32_t af[4];
+                ldmatrix_x4(af, kt_s + tile_off(ka_row, 2 * kk + ka_half));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) Mma<T>::run(sf[nt], af, qf[nt][kk][0], qf[nt][kk][1]);
+            }
+            // sf[nt]: (token g, head 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1)
+            const bool v0 = g < nvalid, v1 = g + 8 < nvalid;
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float p[4];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float x0 = v0 ? sf[nt][j] * a.scale_log2 : -INFINITY;
+                    const float x1 = v1 ? sf[nt][j + 2] * a.scale_log2 : -INFINITY;
+                    float bm = fmaxf(x0, x1);
+                    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+                    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+                    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+                    const float m_new = fmaxf(mrow[nt][j], bm);
+                    const float alpha = fast_exp2(mrow[nt][j] - m_new);
+                    p[j] = fast_exp2(x0 - m_new);
+                    p[j + 2] = fast_exp2(x1 - m_new);
+                    lrow[nt][j] = lrow[nt][j] * alpha + p[j] + p[j + 2];
+                    mrow[nt][j] = m_new;
+#pragma unroll
+                    for (int jj = 0; jj < KS; ++jj) {
+                        acc[nt][jj][j] *= alpha;
+                        acc[nt][jj][j + 2] *= alpha;
+                    }
+                }
+                // P^T rows g / g+8 (heads 2c, 2c+1) -> B fragments of O^T += V^T P^T
+                pb[nt][0] = movmatrix_trans(Mma<T>::pack(p[0], p[1]));
+                pb[nt][1] = movmatrix_trans(Mma<T>::pack(p[2], p[3]));
+            }
+            if (nvalid < kBlock) {
+                // rows past the context may hold anything (NaN included): zero them
+                for (int idx = lane; idx < (kBlock - nvalid) * (D / 8); idx += 32) {
+                    const int t = nvalid + idx / (D / 8), ch = idx % (D / 8);
+                    *reinterpret_cast<uint4 *>(vt + tile_off(t, ch)) = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+#pragma unroll
+            for (int j = 0; j < KS; ++j) {
+                uint32_t af[4];
+                ldmatrix_x4_trans(af, vt_s + tile_off(va_row, 2 * j + va_half));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) Mma<T>::run(acc[nt][j], af, pb[nt][0], pb[nt][1]);
+            }
+        }
+        __syncwarp();
+        if (issued < nk) pipe.issue(issued++);
+    }
+    if (dead) pipe.drain(k, issued);
+
+    // full per-head sums: add the partial sums of the 8 lanes that share c
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float v = lrow[nt][j];
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            lrow[nt][j] = dead ? 0.f : v;
+        }
+    // the warp's ring is idle now: reuse it as [GMAX][D] fp32 scratch
+    float *wacc = reinterpret_cast<float *>(pipe.ring);
+    if (!dead) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < KS; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int h = nt * 8 + 2 * c + (e & 1);
+                    const int d = 16 * j + g + 8 * (e >> 1);
+                    wacc[h * D + d] = acc[nt][j][e];
+                }
+    }
+    if (g == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * c + j;
+                s_m[warp][h] = mrow[nt][j];
+                s_l[warp][h] = lrow[nt][j];
+            }
+    }
+    __syncthreads();
+
+    const uint8_t *rings = align_smem_1024(dyn_smem);
+    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+        const int h = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            if (s_l[w][h] > 0.f) M = fmaxf(M, s_m[w][h]);
+        float den = 0.f, o = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            if (s_l[w][h] > 0.f) {
+                const float wt = fast_exp2(s_m[w][h] - M);
+                den += wt * s_l[w][h];
+                o += wt * reinterpret_cast<const float *>(rings + w * STAGES * Pipe::kStage)[h * D + d];
+            }
+        }
+        o = den > 0.f ? o / den : 0.f;
+        const size_t row = row0 + h;
+        if (nparts == 1) {
+            out[h * D + d] = narrow1(o, T());
+        } else {
+            a.ws_o[(row * a.num_parts + part) * D + d] = o;
+            if (d == 0) a.ws_ml[row * a.num_parts + part] = make_float2(den > 0.f ? M : -INFINITY, den);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ partition merge
+// One CTA of kMergeThreads per (sequence, q head) whose context spans more
+// than one partition: out = sum_p w_p o_p / sum_p w_p, w_p = l_p 2^(m_p - M).
+constexpr int kMergeThreads = 128;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
+    extern __shared__ float s_w[];  // [num_parts]
+    __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float s_bcast;
+    const int row = blockIdx.x;
+    const int s = row / a.num_q_heads;
+    const int L = clamp_context(a, s, false);
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
+    if (nparts <= 1) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float2 *ml = a.ws_ml + (size_t)row * a.num_parts;
+
+    float M = -INFINITY;
+    for (int p = threadIdx.x; p < nparts; p += kMergeThreads) {
+        const float2 v = ml[p];
+        if (v.y > 0.f) M = fmaxf(M, v.x);
+    }
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) s_red[warp] = M;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float v = s_red[0];
+        for (int w = 1; w < kMergeThreads / 32; ++w) v = fmaxf(v, s_red[w]);
+        s_bcast = v;
+    }
+    __syncthreads();
+    M = s_bcast;
+    float den = 0.f;
+    for (int p = threadIdx.x; p < nparts; p += kMergeThreads) {
+        const float2 v = ml[p];
+        const float w = v.y > 0.f ? v.y * fast_exp2(v.x - M) : 0.f;
+        s_w[p] = w;
+        den += w;
+    }
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    __syncthreads();  // s_red reuse
+    if (lane == 0) s_red[warp] = den;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float v = 0.f;
+        for (int w = 0; w < kMergeThreads / 32; ++w) v += s_red[w];
+        s_bcast = v;
+    }
+    __syncthreads();
+    den = s_bcast;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const float *o_parts = a.ws_o + (size_t)row * a.num_parts * D;
+    uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + (size_t)row * D;
+    for (int d = threadIdx.x; d < D; d += kMergeThreads) {
+        float o = 0.f;
+        for (int p = 0; p < nparts; ++p)
+            if (s_w[p] != 0.f) o += s_w[p] * o_parts[(size_t)p * D + d];
+        out[d] = narrow1(o * inv, T());
+    }
+}
+
+// ------------------------------------------------------------------ scatter write
+// One CTA per token: kv head h, 16-byte chunk c of K and V row -> slot.
+template <int D>
+__global__ void scatter_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                               uint4 *__restrict__ kc, uint4 *__restrict__ vc,
+                               const int64_t *__restrict__ slots, int num_kv_heads,
+                               long long num_slots) {
+    constexpr int VPR = D / 8;  // 16-byte vectors per row
+    const int t = blockIdx.x;
+    const long long slot = slots[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0) flag_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const long long b = slot / kBlock, o = slot % kBlock;
+    for (int i = threadIdx.x; i < num_kv_heads * VPR; i += blockDim.x) {
+        const int h = i / VPR, c = i % VPR;
+        const size_t src = ((size_t)t * num_kv_heads + h) * VPR + c;
+        const size_t dst = (((size_t)b * num_kv_heads + h) * kBlock + o) * VPR + c;
+        kc[dst] = k[src];
+        vc[dst] = v[src];
+    }
+}
+
+// ------------------------------------------------------------------ block copy
+// grid.x strides over pairs, grid.y over 16-byte chunks of a block.
+__global__ void copy_blocks_kernel(uint4 *__restrict__ kc, uint4 *__restrict__ vc,
+                                   const int32_t *__restrict__ pairs, int num_pairs,
+                                   long long num_blocks, long long vec_per_block) {
+    for (int p = blockIdx.x; p < num_pairs; p += gridDim.x) {
+        const long long src = pairs[2 * p], dst = pairs[2 * p + 1];
+        if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
+            if (blockIdx.y == 0 && threadIdx.x == 0) flag_error(PA_DEVERR_PAIR);
+            continue;
+        }
+        const uint4 *ks = kc + src * vec_per_block;
+        const uint4 *vs = vc + src * vec_per_block;
+        uint4 *kd = kc + dst * vec_per_block;
+        uint4 *vd = vc + dst * vec_per_block;
+        for (long long i = (long long)blockIdx.y * blockDim.x + threadIdx.x; i < vec_per_block;
+             i += (long long)gridDim.y * blockDim.x) {
+            kd[i] = ks[i];
+            vd[i] = vs[i];
+        }
+    }
+}
+
+}  // namespace pa

@@ -1,0 +1,249 @@
+"""CPU tests of libpa.so: exported symbols, the host block allocator, and the
+capacity arithmetic against the figures the pages print (no GPU needed)."""
+import ctypes
+import json
+import os
+import re
+import shutil
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+pk = pytest.importorskip("paged_kv_cache_425_b200")
+from paged_kv_cache_425_b200 import batch  # noqa: E402
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(pa_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert "pa_decode" in names and "pa_reshape_and_cache" in names and "pa_copy_blocks" in names
+    lib = ctypes.CDLL(pk.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    assert pk.pa_status_string(0) == b"ok"
+    assert pk.pa_status_string(pk.PA_ERR_WORKSPACE).startswith(b"workspace")
+    assert pk.pa_version() >= 100
+
+
+def test_workspace_size_rule():
+    assert pk.decode_workspace_size(64, 32, 128, 32) == 0            # one partition
+    n = pk.decode_workspace_size(64, 32, 128, 128)                  # 4 partitions
+    rows = 64 * 32 * 4
+    assert n >= rows * 128 * 4 + rows * 8 and n % 256 == 0
+    assert pk.decode_workspace_size(64, 32, 128, 128, block_size=32) == 0
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    dst = tmp_path / "paged_kv_cache_425_b200"
+    shutil.copytree(os.path.join(ROOT, "paged_kv_cache_425_b200"), dst,
+                    ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    code = "import paged_kv_cache_425_b200"
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True,
+                       env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode != 0 and "missing" in r.stderr
+
+
+# ---------------------------------------------------------------- allocator semantics
+def test_fresh_pool_hands_out_in_order_and_frees_to_the_back():
+    a = pk.BlockAllocator(8)
+    a.add_seq(1, 33)                       # 3 blocks
+    assert list(a.block_table(1)) == [0, 1, 2]
+    a.add_seq(2, 16)
+    assert list(a.block_table(2)) == [3]
+    a.free_seq(1)
+    a.add_seq(3, 64)                       # 4 blocks: 4..7 first, then the freed ones
+    assert list(a.block_table(3)) == [4, 5, 6, 7]
+    a.add_seq(4, 1)
+    assert list(a.block_table(4)) == [0]
+
+
+def test_exhaustion_fails_without_side_effects():
+    a = pk.BlockAllocator(4)
+    a.add_seq(1, 40)                       # 3 blocks
+    before = a.stats()
+    with pytest.raises(pk.PagedError) as e:
+        a.add_seq(2, 17)                   # needs 2, 1 free
+    assert e.value.status == pk.PA_ERR_NO_BLOCKS
+    assert a.stats() == before
+    a.add_seq(2, 16)
+    a.append_slot(1)                       # 41st token fits in block 2
+    with pytest.raises(pk.PagedError):
+        for _ in range(8):
+            a.append_slot(1)               # token 49 needs a 5th block
+    assert a.num_tokens(1) == 48
+
+
+def test_append_slot_places_tokens_by_the_table():
+    a = pk.BlockAllocator(50)
+    rng = np.random.default_rng(0)
+    for s in range(5):
+        a.add_seq(s, int(rng.integers(0, 40)))
+    for _ in range(200):
+        s = int(rng.integers(0, 5))
+        p = a.num_tokens(s)
+        slot, (src, dst) = a.append_slot(s)
+        assert (src, dst) == (-1, -1)
+        t = a.block_table(s)
+        assert slot == t[p // 16] * 16 + p % 16
+        assert len(t) == (p + 1 + 15) // 16
+
+
+def test_fork_shares_and_first_writers_copy_last_writes_in_place():
+    a = pk.BlockAllocator(20)
+    a.add_seq(0, 40)                       # blocks 0,1,2; block 2 holds 8 tokens
+    for c in (1, 2, 3):
+        a.fork(0, c)
+    assert [a.refcount(b) for b in (0, 1, 2)] == [4, 4, 4]
+    copies = []
+    for s in (0, 1, 2, 3):
+        slot, pair = a.append_slot(s)
+        copies.append(pair)
+        t = a.block_table(s)
+        assert slot == t[2] * 16 + 8
+    assert copies[:3] == [(2, 3), (2, 4), (2, 5)]  # first three writers copy block 2
+    assert copies[3] == (-1, -1)                   # the last holder writes in place
+    assert list(a.block_table(3)) == [0, 1, 2]
+    assert [a.refcount(b) for b in (0, 1, 2, 3, 4, 5)] == [4, 4, 1, 1, 1, 1]
+    st = a.stats()
+    assert st["cow_copies"] == 3 and st["shared_blocks"] == 2
+    # a full shared block needs no copy: the next token opens a new block
+    b = pk.BlockAllocator(10)
+    b.add_seq(0, 32)
+    b.fork(0, 1)
+    _, pair = b.append_slot(1)
+    assert pair == (-1, -1) and b.block_table(1)[2] not in (0, 1)
+
+
+def test_free_releases_only_unshared_blocks():
+    a = pk.BlockAllocator(10)
+    a.add_seq(0, 20)
+    a.fork(0, 1)
+    a.free_seq(0)
+    assert a.stats()["free_blocks"] == 8
+    a.free_seq(1)
+    assert a.stats()["free_blocks"] == 10
+
+
+def test_random_operations_keep_the_pool_consistent():
+    """Refcounts equal the number of tables holding each block; free + used =
+    pool; tables have ceil(tokens / 16) entries."""
+    rng = np.random.default_rng(1)
+    a = pk.BlockAllocator(200)
+    live, next_id = set(), 0
+    for _ in range(3000):
+        op = rng.integers(0, 4)
+        try:
+            if op == 0 or not live:
+                a.add_seq(next_id, int(rng.integers(0, 60)))
+                live.add(next_id)
+                next_id += 1
+            elif op == 1:
+                s = int(rng.choice(sorted(live)))
+                a.fork(s, next_id)
+                live.add(next_id)
+                next_id += 1
+            elif op == 2:
+                a.append_slot(int(rng.choice(sorted(live))))
+            else:
+                s = int(rng.choice(sorted(live)))
+                a.free_seq(s)
+                live.discard(s)
+        except pk.PagedError as e:
+            assert e.status == pk.PA_ERR_NO_BLOCKS
+        holders = np.zeros(200, np.int64)
+        for s in live:
+            t = a.block_table(s)
+            assert len(t) == (a.num_tokens(s) + 15) // 16
+            assert len(set(t.tolist())) == len(t)
+            np.add.at(holders, t, 1)
+        rc = np.array([a.refcount(b) for b in range(200)])
+        assert np.array_equal(rc, holders)
+        st = a.stats()
+        assert st["free_blocks"] + st["used_blocks"] == 200
+        assert st["used_blocks"] == int((rc > 0).sum())
+
+
+def test_build_tables_pads_with_minus_one():
+    a = pk.BlockAllocator(10)
+    a.add_seq(7, 20)
+    a.add_seq(9, 0)
+    t, lens = a.build_tables([9, 7], 4)
+    assert t.tolist() == [[-1, -1, -1, -1], [0, 1, -1, -1]] and lens.tolist() == [0, 20]
+    with pytest.raises(pk.PagedError):
+        a.build_tables([7], 1)
+
+
+# ---------------------------------------------------------------- the pages' figures
+@pytest.mark.parametrize("name", ["llama7b", "llama13b"])
+def test_waste_below_four_percent(name):
+    """Paging wastes at most the tail of each sequence's last block: under 4 %
+    ('vLLM PagedAttention: reducing KV cache memory waste', opening and 'How
+    PagedAttention Works')."""
+    w = wl.WORKLOADS[name]
+    rng = wl.rng_for(0)
+    lens = wl.draw_context_lens(w, rng)
+    nb = wl.pool_size(w, lens)
+    b = batch.decode_batch(w, lens, wl.draw_block_order(nb, rng), nb, batch.max_blocks_for(w))
+    st = b.alloc.stats()
+    last_block_tail = sum((-int(L)) % 16 for L in lens)
+    assert st["filled_slots"] == int(lens.sum())
+    assert st["used_blocks"] * 16 - st["filled_slots"] == last_block_tail
+    assert st["waste"] < 0.04
+    # the tables really are scattered: few consecutive neighbours
+    t = b.tables
+    nxt = (t[:, 1:] == t[:, :-1] + 1) & (t[:, 1:] >= 0)
+    assert nxt.sum() < 0.01 * (t >= 0).sum()
+
+
+def test_copy_on_write_step_of_the_sampling_workload():
+    w = wl.WORKLOADS["cow"]
+    rng = wl.rng_for(0)
+    own = wl.draw_branch_tokens(w, rng)
+    nb = batch.cow_pool_blocks(w)
+    fb = batch.ForkedBatch(w, own, wl.draw_block_order(nb, rng), nb)
+    b = fb.step()
+    assert len(b.pairs) == w.prompts * (w.branches - 1)
+    assert np.all(b.context_lens == w.prompt_len + 1)
+    st = fb.alloc.stats()
+    assert st["shared_blocks"] == w.prompts * (w.prompt_len // 16)
+    assert st["sharing_saving"] > 0.5
+
+
+def test_kv_size_formula_reproduces_printed_13b_figure():
+    with open(os.path.join(GOLDEN, "kv_size_13b.json")) as f:
+        g = json.load(f)
+    per_token = pk.kv_bytes_per_token(g["layers"], g["kv_heads"], g["head_dim"], g["dtype_bytes"])
+    assert per_token == 2 * 40 * 5120 * 2
+    gb = per_token * g["tokens"] / 1e9
+    assert abs(gb - g["printed_gb"]) <= g["printed_gb_tolerance"]
+    assert abs(gb - g["rough_gb"]) <= g["rough_gb_tolerance"]
+
+
+def test_pool_budget_reproduces_printed_figure():
+    with open(os.path.join(GOLDEN, "pool_budget.json")) as f:
+        g = json.load(f)
+    got = pk.pool_bytes(g["gpu_gb"] * 1e9, g["weights_gb"] * 1e9, g["utilization"]) / 1e9
+    assert abs(got - g["printed_pool_gb"]) < 1e-9
+    assert pk.pool_bytes(8e9, 16e9, 0.9) == 0.0
+    blocks = pk.pool_num_blocks(got * 1e9, 32, 8, 128, 16, 2)  # Llama-3.1-8B shape
+    assert blocks == int(7.2e9 // (16 * 2 * 32 * 8 * 128 * 2))

@@ -1,0 +1,291 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Bit-exact for the scatter write and the block copy (whole pool compared);
+attention outputs within max-abs 2e-3 (fp16) / 1e-2 (bf16) of the oracle.
+Sizes span several 16-token blocks, several 512-token partitions and ragged
+tails; edge cases: one token, empty context, identical keys, permuted
+placement, bad indices reported through the device error word.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+from paged_inputs import make_paged, to_f64 as bits_f64
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import gpu_harness as gh  # noqa: E402
+
+pk = pytest.importorskip("paged_kv_cache_425_b200")
+
+
+def oracle_out(p, seqs=None):
+    return oracle.decode(p.q, p.key_cache, p.value_cache, p.tables, p.lens, p.num_kv_heads,
+                         p.scale, p.dtype, seqs=seqs)
+
+
+def gpu_out(p, stream=None):
+    return gh.run_decode(pk, p.q, p.key_cache, p.value_cache, p.tables, p.lens, p.num_kv_heads,
+                         p.scale, p.dtype, stream=stream)
+
+
+# ---------------------------------------------------------------- the tiny workload, whole step
+def test_tiny_workload_step():
+    """4 seqs, 4/4 heads, d 64, fp16, ctx U{1..64}, 64-block pool, one new
+    token per sequence written by pa_reshape_and_cache, then pa_decode."""
+    w = wl.WORKLOADS["tiny"]
+    rng = wl.rng_for(0)
+    lens = wl.draw_context_lens(w, rng)
+    p = make_paged(rng, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, lens,
+                   w.pool_blocks, w.dtype, scale=w.scale)
+    k_new = wl.draw_values(rng, (w.num_seqs, w.num_kv_heads, w.head_dim), w.dtype)
+    v_new = wl.draw_values(rng, (w.num_seqs, w.num_kv_heads, w.head_dim), w.dtype)
+    pos = lens - 1
+    slots = np.array([p.tables[s, pos[s] // 16] * 16 + pos[s] % 16 for s in range(w.num_seqs)],
+                     np.int64)
+    kc, vc = gh.to_dev(p.key_cache, w.dtype), gh.to_dev(p.value_cache, w.dtype)
+    pk.reshape_and_cache(gh.to_dev(k_new, w.dtype), gh.to_dev(v_new, w.dtype), kc, vc,
+                         gh.ints(slots, torch.int64))
+    out = gh.run_decode(pk, p.q, kc, vc, p.tables, p.lens, w.num_kv_heads, w.scale, w.dtype)
+    assert pk.get_error() == (0, 0)
+    oracle.reshape_and_cache(k_new, v_new, p.key_cache, p.value_cache, slots)
+    assert np.array_equal(gh.to_host_bits(kc), p.key_cache)
+    assert np.array_equal(gh.to_host_bits(vc), p.value_cache)
+    assert gh.max_err(out, oracle_out(p)) <= gh.TOL[w.dtype]
+
+
+# ---------------------------------------------------------------- shapes x lengths
+LENS = [1, 15, 16, 17, 100, 511, 512, 513, 1024, 1500, 2049, 3000]
+
+
+@pytest.mark.parametrize("dtype", [wl.F16, wl.BF16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("hq,hkv,d", [(2, 2, 128), (3, 3, 64), (8, 4, 128), (8, 2, 64),
+                                      (16, 4, 128), (8, 1, 128), (12, 1, 64), (16, 1, 128),
+                                      (32, 8, 128)])
+def test_decode_shapes_and_lengths(dtype, hq, hkv, d):
+    rng = wl.rng_for(100 + hq * 7 + hkv + d)
+    lens = np.array(LENS, np.int32)
+    nb = wl.blocks_needed(lens, 16) + 5
+    p = make_paged(rng, len(lens), hq, hkv, d, lens, nb, dtype)
+    err = gh.max_err(gpu_out(p), oracle_out(p))
+    assert err <= gh.TOL[dtype], err
+
+
+@pytest.mark.parametrize("hq,hkv,d,dtype", [(2, 2, 64, wl.F16), (8, 2, 128, wl.BF16),
+                                            (4, 4, 128, wl.BF16)])
+def test_every_context_length_1_to_64(hq, hkv, d, dtype):
+    rng = wl.rng_for(7)
+    lens = np.arange(1, 65, dtype=np.int32)
+    p = make_paged(rng, 64, hq, hkv, d, lens, wl.blocks_needed(lens, 16), dtype)
+    assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[dtype]
+
+
+def test_wide_table_many_partitions():
+    """Table width 2048 blocks (64 partitions) with short and long contexts."""
+    rng = wl.rng_for(8)
+    lens = np.array([5, 8192, 32768, 513, 20000], np.int32)
+    nb = wl.blocks_needed(lens, 16) + 3
+    p = make_paged(rng, 5, 8, 2, 128, lens, nb, wl.BF16, max_blocks=2048)
+    assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[wl.BF16]
+
+
+# ---------------------------------------------------------------- closed forms on the GPU
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2)])
+def test_one_token_returns_v0_exactly(hq, hkv):
+    rng = wl.rng_for(9)
+    p = make_paged(rng, 3, hq, hkv, 128, [1, 1, 1], 3, wl.BF16)
+    out = gh.to_host_bits(gpu_out(p))
+    G = hq // hkv
+    for s in range(3):
+        for h in range(hq):
+            assert np.array_equal(out[s, h], p.v_dense[s, 0, h // G])
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (16, 2)])
+def test_empty_context_gives_zeros(hq, hkv):
+    rng = wl.rng_for(10)
+    p = make_paged(rng, 3, hq, hkv, 64, [0, 700, 0], 50, wl.F16)
+    out = gh.to_f64(gpu_out(p))
+    assert np.all(out[0] == 0) and np.all(out[2] == 0)
+    assert np.max(np.abs(out[1] - oracle_out(p)[1])) <= gh.TOL[wl.F16]
+
+
+def test_identical_keys_give_mean_of_values():
+    rng = wl.rng_for(11)
+    lens = [37, 600, 5]
+    p = make_paged(rng, 3, 8, 2, 128, lens, 60, wl.F16)
+    p.key_cache[:] = p.key_cache[0, 0, 0]
+    out = gh.to_f64(gpu_out(p))
+    for s, L in enumerate(lens):
+        mean = bits_f64(p.v_dense[s, :L], wl.F16).mean(axis=0)  # [Hkv, d]
+        assert np.max(np.abs(out[s] - np.repeat(mean, 4, axis=0))) <= gh.TOL[wl.F16]
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2)])
+def test_physical_placement_is_invisible_bitwise(hq, hkv):
+    """Same logical sequences in a differently ordered pool: identical bits."""
+    lens = np.array([700, 17, 1, 48, 1100], np.int32)
+    nb = wl.blocks_needed(lens, 16)
+    a = make_paged(wl.rng_for(12), 5, hq, hkv, 128, lens, nb, wl.BF16)
+    order = wl.draw_block_order(nb, wl.rng_for(99))
+    from paged_inputs import tables_from_order
+    tb = tables_from_order(lens, order, 16, a.tables.shape[1])
+    kc = np.zeros_like(a.key_cache)
+    vc = np.zeros_like(a.value_cache)
+    for s in range(5):
+        n = (int(lens[s]) + 15) // 16
+        kc[tb[s, :n]] = a.key_cache[a.tables[s, :n]]
+        vc[tb[s, :n]] = a.value_cache[a.tables[s, :n]]
+    ra = gh.to_host_bits(gpu_out(a))
+    rb = gh.to_host_bits(gh.run_decode(pk, a.q, kc, vc, tb, lens, hkv, a.scale, wl.BF16))
+    assert np.array_equal(ra, rb)
+
+
+def test_runs_on_a_side_stream():
+    rng = wl.rng_for(13)
+    lens = np.array([900, 33, 1025], np.int32)
+    p = make_paged(rng, 3, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.F16)
+    s = torch.cuda.Stream()
+    out = gpu_out(p, stream=s)
+    assert gh.max_err(out, oracle_out(p)) <= gh.TOL[wl.F16]
+
+
+# ---------------------------------------------------------------- scatter write / block copy
+@pytest.mark.parametrize("d,dtype", [(64, wl.F16), (128, wl.BF16)])
+def test_reshape_and_cache_bit_exact(d, dtype):
+    rng = wl.rng_for(14)
+    nb, hkv, T = 40, 6, 50
+    kc = wl.draw_values(rng, (nb, hkv, 16, d), dtype)
+    vc = wl.draw_values(rng, (nb, hkv, 16, d), dtype)
+    k = wl.draw_values(rng, (T, hkv, d), dtype)
+    v = wl.draw_values(rng, (T, hkv, d), dtype)
+    slots = rng.choice(nb * 16, size=T, replace=False).astype(np.int64)
+    slots[::7] = -1  # padding entries
+    dkc, dvc = gh.to_dev(kc, dtype), gh.to_dev(vc, dtype)
+    pk.reshape_and_cache(gh.to_dev(k, dtype), gh.to_dev(v, dtype), dkc, dvc,
+                         gh.ints(slots, torch.int64))
+    assert pk.get_error() == (0, 0)
+    assert oracle.reshape_and_cache(k, v, kc, vc, slots) == 0
+    assert np.array_equal(gh.to_host_bits(dkc), kc)
+    assert np.array_equal(gh.to_host_bits(dvc), vc)
+
+
+@pytest.mark.parametrize("d,hkv", [(64, 4), (128, 32)])
+def test_copy_blocks_bit_exact(d, hkv):
+    rng = wl.rng_for(15)
+    nb = 300
+    kc = wl.draw_values(rng, (nb, hkv, 16, d), wl.BF16)
+    vc = wl.draw_values(rng, (nb, hkv, 16, d), wl.BF16)
+    perm = rng.permutation(nb)
+    pairs = np.stack([perm[:96], perm[96:192]], axis=1).astype(np.int32)
+    dkc, dvc = gh.to_dev(kc, wl.BF16), gh.to_dev(vc, wl.BF16)
+    pk.copy_blocks(dkc, dvc, gh.ints(pairs))
+    assert pk.get_error() == (0, 0)
+    oracle.copy_blocks(kc, vc, pairs)
+    assert np.array_equal(gh.to_host_bits(dkc), kc)
+    assert np.array_equal(gh.to_host_bits(dvc), vc)
+
+
+def test_copy_blocks_no_pairs_is_a_no_op():
+    kc = torch.zeros((4, 2, 16, 64), dtype=torch.float16, device="cuda")
+    pk.copy_blocks(kc, kc.clone(), torch.zeros((0, 2), dtype=torch.int32, device="cuda"))
+
+
+# ---------------------------------------------------------------- copy-on-write workload (scaled)
+def test_parallel_sampling_copy_on_write_steps():
+    """Prompts forked into branches through the allocator; every step does the
+    copy-on-write copies, writes one token per live branch and decodes; the
+    pool and outputs match the oracle replaying the same calls."""
+    from paged_kv_cache_425_b200 import batch
+    w = wl.scaled(wl.WORKLOADS["cow"], prompts=4, prompt_len=100, own_max=20, num_seqs=16)
+    rng = wl.rng_for(16)
+    own = wl.draw_branch_tokens(w, rng)
+    nb = batch.cow_pool_blocks(w)
+    fb = batch.ForkedBatch(w, own, wl.draw_block_order(nb, rng), nb)
+    H, d, dt = w.num_kv_heads, w.head_dim, w.dtype
+    kc = wl.draw_values(rng, (nb, H, 16, d), dt)
+    vc = wl.draw_values(rng, (nb, H, 16, d), dt)
+    dkc, dvc = gh.to_dev(kc, dt), gh.to_dev(vc, dt)
+    total_pairs = 0
+    for step in range(fb.num_steps):
+        b = fb.step()
+        n = len(b.seq_ids)
+        q = wl.draw_values(rng, (n, w.num_q_heads, d), dt)
+        k_new = wl.draw_values(rng, (n, H, d), dt)
+        v_new = wl.draw_values(rng, (n, H, d), dt)
+        if len(b.pairs):
+            pk.copy_blocks(dkc, dvc, gh.ints(b.pairs))
+            oracle.copy_blocks(kc, vc, b.pairs)
+            total_pairs += len(b.pairs)
+        pk.reshape_and_cache(gh.to_dev(k_new, dt), gh.to_dev(v_new, dt), dkc, dvc,
+                             gh.ints(b.slots, torch.int64))
+        oracle.reshape_and_cache(k_new, v_new, kc, vc, b.slots)
+        out = gh.run_decode(pk, q, dkc, dvc, b.tables, b.context_lens, H, w.scale, dt)
+        ref = oracle.decode(q, kc, vc, b.tables, b.context_lens, H, w.scale, dt)
+        assert gh.max_err(out, ref) <= gh.TOL[dt], step
+        if step in (0, 1, fb.num_steps - 1):
+            assert np.array_equal(gh.to_host_bits(dkc), kc)
+            assert np.array_equal(gh.to_host_bits(dvc), vc)
+    assert total_pairs == w.prompts * (w.branches - 1)
+    assert pk.get_error() == (0, 0)
+
+
+# ---------------------------------------------------------------- errors
+def test_bad_block_id_is_reported_and_skipped():
+    rng = wl.rng_for(17)
+    lens = np.array([40, 40], np.int32)
+    p = make_paged(rng, 2, 4, 4, 64, lens, 6, wl.F16)
+    ref = oracle_out(p)
+    p.tables[1, 1] = 10_000  # out of the pool
+    out = gpu_out(p)
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_BLOCK_ID
+    assert gh.max_err(out[:1], ref[:1]) <= gh.TOL[wl.F16]  # other sequences unaffected
+    assert np.all(np.isfinite(gh.to_f64(out)))
+    assert pk.get_error() == (0, 0)  # cleared
+
+
+def test_bad_slot_and_pair_are_reported():
+    kc = torch.zeros((4, 2, 16, 64), dtype=torch.float16, device="cuda")
+    vc = torch.zeros_like(kc)
+    k = torch.ones((2, 2, 64), dtype=torch.float16, device="cuda")
+    pk.reshape_and_cache(k, k, kc, vc, torch.tensor([3, 4 * 16], dtype=torch.int64, device="cuda"))
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits == pk.DEVERR_SLOT
+    assert torch.all(kc.view(-1, 64)[3] == 1) and int((kc != 0).sum()) == 2 * 64
+    pk.copy_blocks(kc, vc, torch.tensor([[0, 1], [2, 9]], dtype=torch.int32, device="cuda"))
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits == pk.DEVERR_PAIR
+
+
+def test_context_len_beyond_table_is_reported_and_clamped():
+    rng = wl.rng_for(18)
+    lens = np.array([32, 20], np.int32)
+    p = make_paged(rng, 2, 2, 2, 64, lens, 4, wl.F16, max_blocks=2)
+    ref = oracle_out(p)
+    p.lens = np.array([32, 20 + 1000], np.int32)
+    out = gpu_out(p)
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_CONTEXT_LEN
+    assert gh.max_err(out[:1], ref[:1]) <= gh.TOL[wl.F16]
+
+
+def test_host_side_rejections():
+    q = torch.zeros((2, 4, 96), dtype=torch.float16, device="cuda")
+    kc = torch.zeros((4, 4, 16, 96), dtype=torch.float16, device="cuda")
+    tb = torch.zeros((2, 40), dtype=torch.int32, device="cuda")
+    ln = torch.ones(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(pk.PagedError) as e:
+        pk.decode(q.clone(), q, kc, kc, tb, ln, 4, 0.1)
+    assert e.value.status == pk.PA_ERR_UNSUPPORTED
+    q = torch.zeros((2, 4, 64), dtype=torch.float16, device="cuda")
+    kc = torch.zeros((4, 4, 16, 64), dtype=torch.float16, device="cuda")
+    with pytest.raises(pk.PagedError) as e:  # 40 blocks = 3 partitions, no workspace
+        pk.decode(q.clone(), q, kc, kc, tb, ln, 4, 0.1)
+    assert e.value.status == pk.PA_ERR_WORKSPACE
+    with pytest.raises(pk.PagedError) as e:  # 4 q heads over 3 kv heads
+        kc3 = torch.zeros((4, 3, 16, 64), dtype=torch.float16, device="cuda")
+        pk.decode(q.clone(), q, kc3, kc3, tb[:, :2].contiguous(), ln, 3, 0.1)
+    assert e.value.status == pk.PA_ERR_INVALID_ARG
