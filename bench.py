@@ -26,7 +26,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -54,6 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=0,
                     help="layer caches to allocate (0: the workload's layer count; fewer "
                          "caches are cycled so every step still runs every layer)")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="run the workload with fewer sequences (small profiling case; "
+                         "the bench line then names the reduced size)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -154,50 +156,64 @@ def traffic_per_call(workload: str, calls_bytes: int):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clock and clock-event (throttle) reasons, read through NVML every
+    few milliseconds on a background thread during the timed region."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {  # NVML clocks-event-reason bits that matter for a timing
+        0x8: "hw_slowdown",
+        0x40: "hw_thermal_slowdown",
+        0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap",
+    }
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"pa_clocks_{os.getpid()}.csv")
+    def __init__(self, device, period_s: float = 0.005):
+        self.device = device
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.thread = None
+        self.error = None
 
     def start(self):
+        import threading
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.error = f"nvml unavailable: {e}"
+            return
+        self.stop_flag = threading.Event()
+
+        def loop():
+            while not self.stop_flag.is_set():
+                try:
+                    self.samples.append(float(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)))
+                    bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.reasons |= {n for b, n in self.REASONS.items() if bits & b}
+                except Exception as e:
+                    self.error = str(e)
+                    return
+                self.stop_flag.wait(self.period)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) == 7 and parts[0].replace(".", "").isdigit():
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[0]) for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[3:]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][1]),
-                "reasons": reasons, "samples": len(rows)}
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "not sampled"]}
+        self.stop_flag.set()
+        self.thread.join(5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "sm_mhz_min": min(self.samples)}
 
 
 # ---------------------------------------------------------------- our arm
@@ -210,6 +226,8 @@ class Setup:
         from paged_kv_cache_425_b200 import batch
         self.pk = pk
         w = wl.WORKLOADS[args.workload]
+        if args.num_seqs:
+            w = wl.scaled(w, num_seqs=args.num_seqs)
         self.w = w
         rng = wl.rng_for(args.seed + rank)
         tdt = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
@@ -293,8 +311,7 @@ def run_ours(args, world, rank, local):
     # ---- device-resident timing
     L = st.layers
     dec_ms = []
-    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    sampler = ClockSampler(device)
     barrier(device)
     torch.cuda.synchronize()
     sampler.start()

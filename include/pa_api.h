@@ -74,7 +74,9 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 
 #define PA_BLOCK_SIZE 16
 /* Decode splits a context into partitions of this many tokens (32 blocks). */
+#ifndef PA_PARTITION_TOKENS
 #define PA_PARTITION_TOKENS 512
+#endif
 
 /* Bits of the device error word (pa_get_error). */
 #define PA_DEVERR_BLOCK_ID 1u    /* block table entry outside [0, num_blocks) */

@@ -13,10 +13,20 @@
 namespace pa {
 namespace {
 
-// Decode launch shape: warps per CTA and TMA stages per warp.
-constexpr int kWarps = 4;
-constexpr int kStages128 = 3;  // 3 x 8 KiB per warp at head_dim 128
-constexpr int kStages64 = 4;   // 4 x 4 KiB per warp at head_dim 64
+// Decode launch shape: warps per CTA and TMA stages per warp (build-time
+// overridable for tuning sweeps).
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_STAGES_128
+#define PA_STAGES_128 3  // 3 x 8 KiB per warp at head_dim 128
+#endif
+#ifndef PA_STAGES_64
+#define PA_STAGES_64 4   // 4 x 4 KiB per warp at head_dim 64
+#endif
+constexpr int kWarps = PA_DECODE_WARPS;
+constexpr int kStages128 = PA_STAGES_128;
+constexpr int kStages64 = PA_STAGES_64;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
