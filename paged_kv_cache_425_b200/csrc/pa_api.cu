@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "pa_api.h"
 #include "pa_kernels.cuh"
@@ -19,10 +20,13 @@ namespace {
 #define PA_DECODE_WARPS 4
 #endif
 #ifndef PA_STAGES_128
-#define PA_STAGES_128 3  // 3 x 8 KiB per warp at head_dim 128
+#define PA_STAGES_128 1  // 1 x 8 KiB per warp at head_dim 128: 6 CTAs per SM
 #endif
 #ifndef PA_STAGES_64
-#define PA_STAGES_64 4   // 4 x 4 KiB per warp at head_dim 64
+#define PA_STAGES_64 2   // 2 x 4 KiB per warp at head_dim 64
+#endif
+#ifndef PA_MHA_ON_MMA
+#define PA_MHA_ON_MMA 0  // 1: one query head per kv head also takes the mma.sync kernel
 #endif
 constexpr int kWarps = PA_DECODE_WARPS;
 constexpr int kStages128 = PA_STAGES_128;
@@ -79,7 +83,26 @@ int check_cache_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size
     return PA_OK;
 }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel in the stream finishes; it waits for that kernel
+// (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}
 
 template <typename Kernel>
 bool set_smem(Kernel k, int bytes) {
@@ -92,26 +115,25 @@ int launch_decode(const DecodeArgs &a, int group, const CUtensorMap &tmk, const 
                   cudaStream_t st) {
     constexpr int STAGES = D == 128 ? kStages128 : kStages64;
     constexpr int SMEM = kWarps * STAGES * WarpPipe<D, STAGES>::kStage + 1024;
-    dim3 grid(a.num_parts, a.num_kv_heads, a.num_seqs);
-    dim3 block(kWarps * 32);
-    if (group == 1) {
+    const dim3 grid(a.num_seqs * a.num_kv_heads, a.num_parts);
+    const dim3 block(kWarps * 32);
+    int rc;
+    if (group == 1 && !PA_MHA_ON_MMA) {
         auto k = decode_simt_kernel<T, D, kWarps, STAGES>;
         if (!set_smem(k, SMEM)) return PA_ERR_CUDA;
-        k<<<grid, block, SMEM, st>>>(tmk, tmv, a);
+        rc = launch_pdl(k, grid, block, SMEM, st, tmk, tmv, a);
     } else if (group <= 8) {
         auto k = decode_mma_kernel<T, D, kWarps, STAGES, 1>;
         if (!set_smem(k, SMEM)) return PA_ERR_CUDA;
-        k<<<grid, block, SMEM, st>>>(tmk, tmv, a);
+        rc = launch_pdl(k, grid, block, SMEM, st, tmk, tmv, a);
     } else {
         auto k = decode_mma_kernel<T, D, kWarps, STAGES, 2>;
         if (!set_smem(k, SMEM)) return PA_ERR_CUDA;
-        k<<<grid, block, SMEM, st>>>(tmk, tmv, a);
+        rc = launch_pdl(k, grid, block, SMEM, st, tmk, tmv, a);
     }
-    int rc = launch_status();
     if (rc != PA_OK || a.num_parts <= 1) return rc;
-    merge_kernel<T, D><<<a.num_seqs * a.num_q_heads, kMergeThreads,
-                         a.num_parts * sizeof(float), st>>>(a);
-    return launch_status();
+    return launch_pdl(merge_kernel<T, D>, dim3(a.num_seqs * a.num_q_heads), dim3(kMergeThreads),
+                      a.num_parts * sizeof(float), st, a);
 }
 
 template <typename T>
@@ -123,6 +145,23 @@ int dispatch_decode(const DecodeArgs &a, int head_dim, int group, const CUtensor
 
 int64_t num_parts_for(int32_t max_blocks_per_seq) {
     return (max_blocks_per_seq + kPartBlocks - 1) / kPartBlocks;
+}
+
+// Workspace: partition outputs fp32 [S][Hq][P][D], then (max, sum) float2
+// [S][Hq][P]; each region starts on a 256-byte boundary.
+struct WorkspaceLayout {
+    int64_t o_off, ml_off, total;
+};
+
+WorkspaceLayout workspace_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim,
+                                 int64_t parts) {
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t rows = num_seqs * num_q_heads * parts;
+    WorkspaceLayout l;
+    l.o_off = 0;
+    l.ml_off = up(rows * head_dim * 4);
+    l.total = l.ml_off + up(rows * 8);
+    return l;
 }
 
 }  // namespace
@@ -146,18 +185,13 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
         return PA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const long long num_slots = num_blocks * kBlock;
-    const int threads = 256;
-    if (head_dim == 128)
-        scatter_kernel<128><<<num_tokens, threads, 0, st>>>(
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-            static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), slot_mapping,
-            num_kv_heads, num_slots);
-    else
-        scatter_kernel<64><<<num_tokens, threads, 0, st>>>(
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-            static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), slot_mapping,
-            num_kv_heads, num_slots);
-    return launch_status();
+    const int vectors = num_kv_heads * (head_dim / 8);
+    const dim3 grid(num_tokens, (vectors + kScatterThreads - 1) / kScatterThreads);
+    if (grid.y > 65535) return PA_ERR_UNSUPPORTED;
+    return launch_pdl(head_dim == 128 ? scatter_kernel<128> : scatter_kernel<64>, grid,
+                      dim3(kScatterThreads), 0, st, static_cast<const uint4 *>(k),
+                      static_cast<const uint4 *>(v), static_cast<uint4 *>(key_cache),
+                      static_cast<uint4 *>(value_cache), slot_mapping, num_kv_heads, num_slots);
 }
 
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
@@ -167,11 +201,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
         return 0;
     const int64_t parts = num_parts_for(max_blocks_per_seq);
     if (parts <= 1) return 0;
-    const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
-    // partition outputs, then (max, sum) pairs, each 256-byte aligned
-    const int64_t o_bytes = (rows * head_dim * 4 + 255) / 256 * 256;
-    const int64_t ml_bytes = (rows * 8 + 255) / 256 * 256;
-    return (size_t)(o_bytes + ml_bytes);
+    return (size_t)workspace_layout(num_seqs, num_q_heads, head_dim, parts).total;
 }
 
 int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
@@ -186,7 +216,7 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     const int group = num_q_heads / num_kv_heads;
     if (group > 16) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PA_OK;
-    if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * num_q_heads >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
         return PA_ERR_INVALID_ARG;
     if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || !aligned(q, 8) ||
@@ -214,10 +244,10 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
                                                      max_blocks_per_seq);
         if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
             return PA_ERR_WORKSPACE;
-        const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
-        const int64_t o_bytes = (rows * head_dim * 4 + 255) / 256 * 256;
-        a.ws_o = static_cast<float *>(workspace);
-        a.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + o_bytes);
+        const WorkspaceLayout l = workspace_layout(num_seqs, num_q_heads, head_dim, parts);
+        char *base = static_cast<char *>(workspace);
+        a.ws_o = reinterpret_cast<float *>(base + l.o_off);
+        a.ws_ml = reinterpret_cast<float2 *>(base + l.ml_off);
     }
     CUtensorMap tmk, tmv;
     if (!encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
@@ -243,10 +273,10 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pa
     long long chunks = (vec_per_block + threads * 4 - 1) / (threads * 4);
     if (chunks > 65535) chunks = 65535;
     dim3 grid(num_pairs < 65535 ? num_pairs : 65535, (unsigned)chunks);
-    copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), src_dst_pairs,
-        num_pairs, num_blocks, vec_per_block);
-    return launch_status();
+    return launch_pdl(copy_blocks_kernel, grid, dim3(threads), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<uint4 *>(key_cache),
+                      static_cast<uint4 *>(value_cache), src_dst_pairs, num_pairs, num_blocks,
+                      vec_per_block);
 }
 
 int pa_get_error(void *stream, uint32_t *bits) {

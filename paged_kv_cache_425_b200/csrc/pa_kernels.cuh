@@ -1,16 +1,19 @@
 // Kernels of the paged KV-cache hot path for B200 (sm_100a).
 //
-//  * scatter_kernel      - pa_reshape_and_cache: one CTA per new token,
-//                          16-byte vectors, K and V rows to their slot.
+//  * scatter_kernel      - pa_reshape_and_cache: one thread per 16-byte
+//                          vector of a new token's K and V rows.
 //  * copy_blocks_kernel  - pa_copy_blocks: 16-byte vector copy of whole
 //                          blocks (all kv heads, K and V).
 //  * decode_simt_kernel  - pa_decode with one query head per kv head.
 //  * decode_mma_kernel   - pa_decode with 2..16 query heads per kv head: the
 //                          query group is one mma.sync tile against each
 //                          16-token K / V tile.
-//  * merge_kernel        - log-sum-exp merge of context partitions.
+//  * merge_kernel        - log-sum-exp merge of the partitions of contexts
+//                          longer than one partition.
 //
-// Decode grid: (partition, kv head, sequence).  A partition covers
+// Decode grid: x = sequence * Hkv + kv head, y = partition (slowest, so the
+// CTAs of partitions past a short sequence's end, which exit at once, come
+// last and overlap the tail of the grid).  A partition covers
 // PA_PARTITION_TOKENS tokens (32 blocks).  Inside a CTA each warp owns every
 // NW-th block of the partition and runs its own STAGES-deep TMA pipeline:
 // one lane loads the warp's next (block, kv head) K and V tiles with
@@ -19,6 +22,12 @@
 // running (max, sum, accumulator) online softmax in fp32, log2 domain.  At
 // the end the CTA combines its warps; a single-partition sequence writes
 // `out`, a split one writes (o, max, sum) to the workspace for merge_kernel.
+//
+// The kernels are chained with programmatic dependent launch: each kernel
+// lets the next one in the stream be scheduled early
+// (griddepcontrol.launch_dependents) and waits for the previous one to
+// complete before touching global memory (griddepcontrol.wait), which hides
+// launch gaps between the scatter, decode and merge kernels.
 //
 // Tile layout in shared memory (matches the TMA 128-byte swizzle): a 16 x D
 // tile is stored as D/64 sub-tiles of 16 rows x 128 bytes; the 16-byte chunk
@@ -101,6 +110,16 @@ __device__ __forceinline__ float reduce16_scatter(float (&v)[16], int lane) {
     return v[0] + __shfl_xor_sync(FULL, v[0], 1);
 }
 
+// Programmatic dependent launch: let the next kernel in the stream be
+// scheduled, and wait until the previous kernel has completed and its memory
+// is visible.  Both are no-ops when the launch has no such dependency.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prior() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Per-warp TMA pipeline over the warp's blocks of one partition.
 template <int D, int STAGES>
 struct WarpPipe {
@@ -174,8 +193,11 @@ __global__ void __launch_bounds__(NW * 32)
     __shared__ __align__(16) float s_acc[NW][D];
     __shared__ float s_m[NW], s_l[NW];
 
-    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int part = blockIdx.y, kvh = blockIdx.x % a.num_kv_heads,
+              s = blockIdx.x / a.num_kv_heads;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_launch_dependents();
+    pdl_wait_prior();
     const int L = clamp_context(a, s, part == 0 && kvh == 0 && threadIdx.x == 0);
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
@@ -362,9 +384,12 @@ __global__ void __launch_bounds__(NW * 32)
     __shared__ __align__(8) uint64_t bars[NW][STAGES];
     __shared__ float s_m[NW][GMAX], s_l[NW][GMAX];
 
-    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int part = blockIdx.y, kvh = blockIdx.x % a.num_kv_heads,
+              s = blockIdx.x / a.num_kv_heads;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.num_q_heads / a.num_kv_heads;
+    pdl_launch_dependents();
+    pdl_wait_prior();
     const int L = clamp_context(a, s, part == 0 && kvh == 0 && threadIdx.x == 0);
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
@@ -574,7 +599,9 @@ __global__ void __launch_bounds__(NW * 32)
 
 // ------------------------------------------------------------------ partition merge
 // One CTA of kMergeThreads per (sequence, q head) whose context spans more
-// than one partition: out = sum_p w_p o_p / sum_p w_p, w_p = l_p 2^(m_p - M).
+// than one partition: out = sum_p w_p o_p / sum_p w_p, w_p = l_p 2^(m_p - M),
+// M = max over partitions that saw a token.  Weights go to shared memory
+// first; the partial outputs then stream in as independent coalesced loads.
 constexpr int kMergeThreads = 128;
 
 template <typename T, int D>
@@ -582,6 +609,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     extern __shared__ float s_w[];  // [num_parts]
     __shared__ float s_red[kMergeThreads / 32];
     __shared__ float s_bcast;
+    pdl_launch_dependents();
+    pdl_wait_prior();
     const int row = blockIdx.x;
     const int s = row / a.num_q_heads;
     const int L = clamp_context(a, s, false);
@@ -614,7 +643,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
         den += w;
     }
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    __syncthreads();  // s_red reuse
+    __syncthreads();  // every thread has read s_bcast; s_red is free again
     if (lane == 0) s_red[warp] = den;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -629,35 +658,41 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + (size_t)row * D;
     for (int d = threadIdx.x; d < D; d += kMergeThreads) {
         float o = 0.f;
-        for (int p = 0; p < nparts; ++p)
-            if (s_w[p] != 0.f) o += s_w[p] * o_parts[(size_t)p * D + d];
+#pragma unroll 8
+        for (int p = 0; p < nparts; ++p) o += s_w[p] * o_parts[(size_t)p * D + d];
         out[d] = narrow1(o * inv, T());
     }
 }
 
 // ------------------------------------------------------------------ scatter write
-// One CTA per token: kv head h, 16-byte chunk c of K and V row -> slot.
+// grid (token, chunk): each thread moves one 16-byte vector of the token's K
+// rows and one of its V rows (vector i = kv head i / (D/8), piece i % (D/8)).
+constexpr int kScatterThreads = 128;
+
 template <int D>
-__global__ void scatter_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
-                               uint4 *__restrict__ kc, uint4 *__restrict__ vc,
-                               const int64_t *__restrict__ slots, int num_kv_heads,
-                               long long num_slots) {
+__global__ void __launch_bounds__(kScatterThreads)
+    scatter_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                   uint4 *__restrict__ kc, uint4 *__restrict__ vc,
+                   const int64_t *__restrict__ slots, int num_kv_heads, long long num_slots) {
     constexpr int VPR = D / 8;  // 16-byte vectors per row
     const int t = blockIdx.x;
+    const int i = blockIdx.y * kScatterThreads + threadIdx.x;
+    pdl_launch_dependents();
+    pdl_wait_prior();
     const long long slot = slots[t];
     if (slot < 0) return;
     if (slot >= num_slots) {
-        if (threadIdx.x == 0) flag_error(PA_DEVERR_SLOT);
+        if (blockIdx.y == 0 && threadIdx.x == 0) flag_error(PA_DEVERR_SLOT);
         return;
     }
+    if (i >= num_kv_heads * VPR) return;
     const long long b = slot / kBlock, o = slot % kBlock;
-    for (int i = threadIdx.x; i < num_kv_heads * VPR; i += blockDim.x) {
-        const int h = i / VPR, c = i % VPR;
-        const size_t src = ((size_t)t * num_kv_heads + h) * VPR + c;
-        const size_t dst = (((size_t)b * num_kv_heads + h) * kBlock + o) * VPR + c;
-        kc[dst] = k[src];
-        vc[dst] = v[src];
-    }
+    const int h = i / VPR, c = i % VPR;
+    const size_t src = (size_t)t * num_kv_heads * VPR + i;
+    const size_t dst = (((size_t)b * num_kv_heads + h) * kBlock + o) * VPR + c;
+    const uint4 kv = k[src], vv = v[src];
+    kc[dst] = kv;
+    vc[dst] = vv;
 }
 
 // ------------------------------------------------------------------ block copy
@@ -665,6 +700,8 @@ __global__ void scatter_kernel(const uint4 *__restrict__ k, const uint4 *__restr
 __global__ void copy_blocks_kernel(uint4 *__restrict__ kc, uint4 *__restrict__ vc,
                                    const int32_t *__restrict__ pairs, int num_pairs,
                                    long long num_blocks, long long vec_per_block) {
+    pdl_launch_dependents();
+    pdl_wait_prior();
     for (int p = blockIdx.x; p < num_pairs; p += gridDim.x) {
         const long long src = pairs[2 * p], dst = pairs[2 * p + 1];
         if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
