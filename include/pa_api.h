@@ -156,6 +156,47 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
                                 int32_t block_size, int32_t max_blocks_per_seq);
 
 /*
+ * pa_decode_static_workspace - pa_decode for callers that cannot allocate.
+ *
+ * The pages have no counterpart for this call: it is an interface
+ * convenience of this library, not a step of the method.
+ *
+ * pa_decode needs split-context scratch (its `workspace`) whenever a context
+ * can span more than one partition.  Some callers cannot hand it over:
+ *  - a serving process that reserves nearly all device memory up front for
+ *    its own KV block pool and weights, so any later cudaMalloc fails or
+ *    fragments that reservation;
+ *  - a hot decode loop that must not call cudaMalloc, because it can
+ *    synchronise the device and stall every stream;
+ *  - a caller in another language that reaches this library through the C
+ *    ABI and has no device allocator of its own.
+ * This entry point computes exactly what pa_decode computes, with the same
+ * arguments minus the workspace.  Its scratch is a fixed array of
+ * PA_STATIC_WORKSPACE_BYTES in the library's device memory: every GPU that
+ * loads the library holds it until the process exits.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Limits and rules:
+ *  - If pa_decode_workspace_size(...) for these sizes exceeds
+ *    PA_STATIC_WORKSPACE_BYTES, the call returns PA_ERR_WORKSPACE and
+ *    enqueues nothing.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current).  Make that first call before any
+ *    stream capture begins.
+ *  - All calls share the one array, and it keeps the last call's contents.
+ *    Nothing in it has to start at zero.  Calls that overlap on the GPU
+ *    (other streams, other host threads) race on the array and give wrong
+ *    results: serialise them.
+ */
+#define PA_STATIC_WORKSPACE_BYTES ((size_t)48 << 20)
+int pa_decode_static_workspace(void *out, const void *q, const void *key_cache,
+                               const void *value_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, int32_t num_kv_heads, float scale,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                               int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+                               int32_t dtype, void *stream);
+
+/*
  * pa_copy_blocks - copy-on-write block copies.
  *
  * Source: "Inside vLLM ...", section "Copy-on-Write Makes Beam Search Cheap";

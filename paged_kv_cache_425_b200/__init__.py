@@ -5,7 +5,7 @@ have the documented shape, type and device, then calls the C entry point of
 the same name (include/pa_api.h, include/pa_alloc.h).  Every step of the hot
 path runs in the library's CUDA kernels; there is no CPU fallback, and
 importing this package fails if the library has not been built
-(``python -m paged_kv_cache_425_b200.build``).
+(``python paged_kv_cache_425_b200/build.py``).
 
 PyTorch serves only as the owner of device memory and streams.
 """
@@ -23,6 +23,7 @@ F16 = 0
 BF16 = 1
 BLOCK_SIZE = 16
 PARTITION_TOKENS = 512
+STATIC_WORKSPACE_BYTES = 48 << 20  # PA_STATIC_WORKSPACE_BYTES
 
 PA_OK = 0
 PA_ERR_INVALID_ARG = -1
@@ -41,7 +42,7 @@ DEVERR_TIMEOUT = 16
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m paged_kv_cache_425_b200.build` (no CPU fallback exists)")
+                      "`python paged_kv_cache_425_b200/build.py` (no CPU fallback exists)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -68,6 +69,8 @@ pa_reshape_and_cache = _sig("pa_reshape_and_cache", ctypes.c_int, _P, _P, _P, _P
 pa_decode = _sig("pa_decode", ctypes.c_int, _P, _P, _P, _P, _P, _P, _i32, _f32, _i32, _i32, _i32,
                  _i32, _i32, _i64, _i32, _P, _sz, _P)
 pa_decode_workspace_size = _sig("pa_decode_workspace_size", _sz, _i32, _i32, _i32, _i32, _i32)
+pa_decode_static_workspace = _sig("pa_decode_static_workspace", ctypes.c_int, _P, _P, _P, _P, _P,
+                                  _P, _i32, _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
 pa_copy_blocks = _sig("pa_copy_blocks", ctypes.c_int, _P, _P, _P, _i32, _i32, _i32, _i32, _i64,
                       _i32, _P)
 pa_get_error = _sig("pa_get_error", ctypes.c_int, _P, ctypes.POINTER(ctypes.c_uint32))
@@ -186,6 +189,31 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, num_kv_he
                      _dev(context_lens, "context_lens", torch.int32, 1), hkv, float(scale), S, hq,
                      d, bs, maxb, nb, dtype_code(q), ws_ptr, ws_bytes, _stream(stream)),
            "pa_decode")
+
+
+def decode_static_workspace(out, q, key_cache, value_cache, block_tables, context_lens,
+                            num_kv_heads: int, scale: float, stream=None):
+    """pa_decode without a workspace argument, for callers that cannot allocate
+    device memory (their memory is reserved up front by their own pools, or
+    the call sits in a loop that must not call cudaMalloc).  The split-context
+    scratch is a fixed array of STATIC_WORKSPACE_BYTES inside the library;
+    larger problems raise PagedError(PA_ERR_WORKSPACE).  Calls sharing the
+    array must not overlap on the GPU."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_shape(key_cache, value_cache)
+    if hkv != num_kv_heads:
+        raise ValueError("num_kv_heads does not match the cache")
+    S, hq, dq = q.shape
+    if dq != d or tuple(out.shape) != (S, hq, d) or out.dtype != q.dtype or q.dtype != key_cache.dtype:
+        raise ValueError("q / out must be [S, Hq, d] of the cache dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    _check(pa_decode_static_workspace(
+        _dev(out, "out"), _dev(q, "q"), _dev(key_cache, "key_cache"),
+        _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables", torch.int32, 2),
+        _dev(context_lens, "context_lens", torch.int32, 1), hkv, float(scale), S, hq, d, bs,
+        int(block_tables.shape[1]), nb, dtype_code(q), _stream(stream)),
+        "pa_decode_static_workspace")
 
 
 def copy_blocks(key_cache, value_cache, src_dst_pairs, stream=None):

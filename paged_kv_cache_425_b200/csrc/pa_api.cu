@@ -308,3 +308,53 @@ const char *pa_status_string(int status) {
 int pa_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation decode
+// Scratch of pa_decode_static_workspace, for callers that cannot allocate
+// device memory (see include/pa_api.h).  In host code `g_static_workspace`
+// names a host-side stand-in, not a device address: its device address is
+// looked up with cudaGetSymbolAddress, once per device, with that device
+// current.
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void *g_static_address[kMaxDevices] = {};
+
+int static_workspace_address(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    if (!g_static_address[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return PA_ERR_CUDA;
+        g_static_address[dev] = p;
+    }
+    *out = g_static_address[dev];
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_decode_static_workspace(void *out, const void *q, const void *key_cache,
+                                          const void *value_cache, const int32_t *block_tables,
+                                          const int32_t *context_lens, int32_t num_kv_heads,
+                                          float scale, int32_t num_seqs, int32_t num_q_heads,
+                                          int32_t head_dim, int32_t block_size,
+                                          int32_t max_blocks_per_seq, int64_t num_blocks,
+                                          int32_t dtype, void *stream) {
+    const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, block_size,
+                                                 max_blocks_per_seq);
+    if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if (need > 0) {
+        const int rc = static_workspace_address(&ws);
+        if (rc != PA_OK) return rc;
+    }
+    return pa_decode(out, q, key_cache, value_cache, block_tables, context_lens, num_kv_heads,
+                     scale, num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, dtype, ws, need > 0 ? PA_STATIC_WORKSPACE_BYTES : 0, stream);
+}
