@@ -1,6 +1,9 @@
 """Build libpa.so in-tree with nvcc for sm_100a.
 
-    python -m paged_kv_cache_425_b200.build [--force] [--ptxas-verbose]
+    python paged_kv_cache_425_b200/build.py [--force] [--ptxas-verbose]
+
+(Run it by path: importing the package itself loads the library this script
+builds.)
 
 The library holds the CUDA kernels, the C ABI of include/pa_api.h and the
 host block allocator of include/pa_alloc.h.  It links the CUDA runtime
