@@ -11,6 +11,10 @@
  *    one prompt share its blocks by reference count; only a branch that
  *    writes into a shared block gets a copy of that block, the rest stays
  *    shared.
+ *  - same page, section "PagedAttention in a Python RAG Application", and its
+ *    question "How does prefix caching work in vLLM and when does it actually
+ *    help?": the content of each block is hashed, and a request whose prefix
+ *    matches reuses the cached physical blocks instead of recomputing them.
  *  - same page, section "Python LLM Inference Optimization with vLLM:
  *    Parameters That Actually Matter": the block pool takes a fraction
  *    (gpu_memory_utilization) of the memory left after the weights.
@@ -48,6 +52,9 @@ typedef struct {
     int64_t logical_blocks; /* sum of the sequences' table lengths */
     int64_t filled_slots;   /* slots of used blocks that hold a token */
     int64_t cow_copies;     /* copy pairs emitted since creation */
+    int64_t cached_blocks;  /* full blocks findable by content (prefix caching) */
+    int64_t prefix_query_blocks; /* full prompt blocks looked up since creation */
+    int64_t prefix_hit_blocks;   /* of those, found in the cache and shared */
     double usage;           /* used_blocks / num_blocks */
     double waste;           /* 1 - filled_slots / (used_blocks * block_size) */
     double sharing_saving;  /* 1 - used_blocks / logical_blocks */
@@ -103,6 +110,29 @@ int32_t pa_alloc_block_table(const pa_alloc *a, int64_t seq_id, int32_t *out, in
  * count.  PA_ERR_INVALID_ARG if a table is longer than max_blocks. */
 int pa_alloc_build_tables(const pa_alloc *a, const int64_t *seq_ids, int32_t n, int32_t *tables,
                           int32_t max_blocks, int32_t *context_lens);
+
+/* Automatic prefix caching on (enable != 0) or off.  When on, every full
+ * block of a prompt added with pa_alloc_add_seq_tokens is registered under a
+ * chain hash of its token ids and of all the tokens before it (64-bit FNV-1a
+ * over the previous block's hash and this block's ids).  A registered block
+ * keeps its place in the cache after its last holder frees it: it goes to
+ * the back of the free list and stays findable until the free list hands it
+ * out again (first in, first out = least recently released first).  Turning
+ * caching off forgets every registration. */
+int pa_alloc_enable_prefix_caching(pa_alloc *a, int32_t enable);
+
+/* pa_alloc_add_seq for a prompt whose token ids are known.  With prefix
+ * caching on, the longest run of leading full blocks whose chain hash and
+ * token ids match registered blocks is shared (refcount + 1; a cached block
+ * on the free list leaves it) instead of claimed, and the blocks claimed for
+ * the remaining full blocks are registered.  *num_cached_tokens receives the
+ * number of leading tokens whose K/V are already in the cache (a multiple of
+ * block_size); the caller writes K/V only for the tokens after them.  The
+ * partly filled last block is never shared.  Without prefix caching this is
+ * pa_alloc_add_seq with *num_cached_tokens = 0.  PA_ERR_NO_BLOCKS (nothing
+ * changed) if the free list cannot serve the blocks that are not cached. */
+int pa_alloc_add_seq_tokens(pa_alloc *a, int64_t seq_id, const int32_t *tokens,
+                            int32_t num_tokens, int32_t *num_cached_tokens);
 
 /* Current reference count of a physical block (0 = free), or -1. */
 int32_t pa_alloc_refcount(const pa_alloc *a, int32_t block);

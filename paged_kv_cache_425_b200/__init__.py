@@ -61,7 +61,9 @@ class AllocStats(ctypes.Structure):
     _fields_ = [("num_blocks", _i64), ("free_blocks", _i64), ("used_blocks", _i64),
                 ("shared_blocks", _i64), ("num_seqs", _i64), ("logical_tokens", _i64),
                 ("logical_blocks", _i64), ("filled_slots", _i64), ("cow_copies", _i64),
-                ("usage", _f64), ("waste", _f64), ("sharing_saving", _f64)]
+                ("cached_blocks", _i64), ("prefix_query_blocks", _i64),
+                ("prefix_hit_blocks", _i64), ("usage", _f64), ("waste", _f64),
+                ("sharing_saving", _f64)]
 
 
 pa_reshape_and_cache = _sig("pa_reshape_and_cache", ctypes.c_int, _P, _P, _P, _P, _P, _i32, _i32,
@@ -89,6 +91,9 @@ pa_alloc_num_tokens = _sig("pa_alloc_num_tokens", _i32, _P, _i64)
 pa_alloc_block_table = _sig("pa_alloc_block_table", _i32, _P, _i64, _P, _i32)
 pa_alloc_build_tables = _sig("pa_alloc_build_tables", ctypes.c_int, _P, _P, _i32, _P, _i32, _P)
 pa_alloc_refcount = _sig("pa_alloc_refcount", _i32, _P, _i32)
+pa_alloc_enable_prefix_caching = _sig("pa_alloc_enable_prefix_caching", ctypes.c_int, _P, _i32)
+pa_alloc_add_seq_tokens = _sig("pa_alloc_add_seq_tokens", ctypes.c_int, _P, _i64, _P, _i32,
+                               ctypes.POINTER(_i32))
 pa_alloc_get_stats = _sig("pa_alloc_get_stats", ctypes.c_int, _P, ctypes.POINTER(AllocStats))
 pa_kv_bytes_per_token = _sig("pa_kv_bytes_per_token", _i64, _i32, _i32, _i32, _i32)
 pa_pool_bytes = _sig("pa_pool_bytes", _f64, _f64, _f64, _f64)
@@ -254,6 +259,19 @@ class BlockAllocator:
 
     def add_seq(self, seq_id: int, num_tokens: int):
         _check(pa_alloc_add_seq(self._h, seq_id, num_tokens), "pa_alloc_add_seq")
+
+    def enable_prefix_caching(self, enable: bool = True):
+        _check(pa_alloc_enable_prefix_caching(self._h, int(bool(enable))),
+               "pa_alloc_enable_prefix_caching")
+
+    def add_seq_tokens(self, seq_id: int, tokens) -> int:
+        """Add a prompt by its token ids; returns how many leading tokens are
+        already cached (their K/V need not be written again)."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        cached = _i32(0)
+        _check(pa_alloc_add_seq_tokens(self._h, seq_id, t.ctypes.data if t.size else None,
+                                       int(t.size), ctypes.byref(cached)), "pa_alloc_add_seq_tokens")
+        return cached.value
 
     def fork(self, parent_id: int, child_id: int):
         _check(pa_alloc_fork(self._h, parent_id, child_id), "pa_alloc_fork")

@@ -1,16 +1,19 @@
 // Host block allocator for the paged KV cache: a first-in-first-out free
-// list, per-block reference counts, per-sequence block tables, and
-// copy-on-write when a sequence writes into a block it shares.
+// list, per-block reference counts, per-sequence block tables,
+// copy-on-write when a sequence writes into a block it shares, and
+// automatic prefix caching of full prompt blocks.
 //
 // Follows "Inside vLLM: How PagedAttention Changes Python LLM Inference at
 // the Systems Level", sections "PagedAttention: What the OS Figured Out
 // Decades Ago" (blocks claimed on demand, released when a sequence ends, a
-// block table per sequence) and "Copy-on-Write Makes Beam Search Cheap"
-// (shared prefix blocks by refcount; only the written block is copied).
+// block table per sequence), "Copy-on-Write Makes Beam Search Cheap" (shared
+// prefix blocks by refcount; only the written block is copied) and
+// "PagedAttention in a Python RAG Application" (the content of each block is
+// hashed; a request whose prefix matches reuses the cached physical blocks).
 // The interface is documented in include/pa_alloc.h.
 #include <cmath>
 #include <cstdint>
-#include <deque>
+#include <cstring>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -25,24 +28,72 @@ struct Sequence {
     int32_t num_tokens = 0;
 };
 
+// 64-bit FNV-1a over a byte string, continued from `h`.
+uint64_t fnv1a(uint64_t h, const void *data, size_t n) {
+    const unsigned char *p = static_cast<const unsigned char *>(data);
+    for (size_t i = 0; i < n; ++i) {
+        h ^= p[i];
+        h *= 1099511628211ull;
+    }
+    return h;
+}
+constexpr uint64_t kFnvOffset = 1469598103934665603ull;
+
 }  // namespace
 
 struct pa_alloc {
     int32_t num_blocks = 0;
     int32_t block_size = 0;
-    std::deque<int32_t> free_list;
+    // free list: intrusive doubly linked list in block order of release, so a
+    // cached block can leave it from the middle in O(1)
+    std::vector<int32_t> next, prev;
+    std::vector<char> in_free;
+    int32_t head = -1, tail = -1;
+    int64_t free_count = 0;
     std::vector<int32_t> refcount;
     std::unordered_map<int64_t, Sequence> seqs;
     int64_t cow_copies = 0;
+    // prefix cache: chain hash of a full block -> block; per block its hash
+    // and token ids (compared on every hit, so a hash collision cannot alias)
+    bool prefix_caching = false;
+    std::unordered_map<uint64_t, int32_t> cached;
+    std::vector<uint64_t> block_hash;
+    std::vector<char> registered;
+    std::vector<int32_t> block_tokens;  // [num_blocks][block_size]
+    int64_t prefix_query_blocks = 0, prefix_hit_blocks = 0;
 
+    void push_back_free(int32_t b) {
+        next[b] = -1;
+        prev[b] = tail;
+        if (tail >= 0) next[tail] = b; else head = b;
+        tail = b;
+        in_free[b] = 1;
+        ++free_count;
+    }
+    void unlink_free(int32_t b) {
+        if (prev[b] >= 0) next[prev[b]] = next[b]; else head = next[b];
+        if (next[b] >= 0) prev[next[b]] = prev[b]; else tail = prev[b];
+        next[b] = prev[b] = -1;
+        in_free[b] = 0;
+        --free_count;
+    }
+    void unregister(int32_t b) {
+        if (!registered[b]) return;
+        auto it = cached.find(block_hash[b]);
+        if (it != cached.end() && it->second == b) cached.erase(it);
+        registered[b] = 0;
+    }
+    // Hand out the block at the front of the free list; a cached block that
+    // comes up is evicted (its contents will be overwritten).
     int32_t claim() {
-        int32_t b = free_list.front();
-        free_list.pop_front();
+        const int32_t b = head;
+        unlink_free(b);
+        unregister(b);
         refcount[b] = 1;
         return b;
     }
     void release(int32_t b) {
-        if (--refcount[b] == 0) free_list.push_back(b);
+        if (--refcount[b] == 0) push_back_free(b);
     }
     int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
 };
@@ -56,7 +107,12 @@ pa_alloc *pa_alloc_create(int32_t num_blocks, int32_t block_size) {
     a->num_blocks = num_blocks;
     a->block_size = block_size;
     a->refcount.assign(num_blocks, 0);
-    for (int32_t b = 0; b < num_blocks; ++b) a->free_list.push_back(b);
+    a->next.assign(num_blocks, -1);
+    a->prev.assign(num_blocks, -1);
+    a->in_free.assign(num_blocks, 0);
+    a->block_hash.assign(num_blocks, 0);
+    a->registered.assign(num_blocks, 0);
+    for (int32_t b = 0; b < num_blocks; ++b) a->push_back_free(b);
     return a;
 }
 
@@ -65,7 +121,7 @@ void pa_alloc_destroy(pa_alloc *a) { delete a; }
 int pa_alloc_add_seq(pa_alloc *a, int64_t seq_id, int32_t num_tokens) {
     if (!a || num_tokens < 0 || a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
     int64_t need = a->blocks_for(num_tokens);
-    if (need > (int64_t)a->free_list.size()) return PA_ERR_NO_BLOCKS;
+    if (need > a->free_count) return PA_ERR_NO_BLOCKS;
     Sequence s;
     s.num_tokens = num_tokens;
     s.blocks.reserve(need);
@@ -96,13 +152,13 @@ int pa_alloc_append_slot(pa_alloc *a, int64_t seq_id, int64_t *slot, int32_t *co
     *cow_dst = -1;
     if (logical == (int32_t)s.blocks.size()) {
         // position p opens a new block
-        if (a->free_list.empty()) return PA_ERR_NO_BLOCKS;
+        if (a->free_count == 0) return PA_ERR_NO_BLOCKS;
         s.blocks.push_back(a->claim());
     } else {
         int32_t last = s.blocks[logical];
         if (a->refcount[last] > 1) {
             // writing into a block others still read: copy it first
-            if (a->free_list.empty()) return PA_ERR_NO_BLOCKS;
+            if (a->free_count == 0) return PA_ERR_NO_BLOCKS;
             int32_t fresh = a->claim();
             a->release(last);
             s.blocks[logical] = fresh;
@@ -187,7 +243,7 @@ int pa_alloc_get_stats(const pa_alloc *a, pa_alloc_stats *out) {
     if (!a || !out) return PA_ERR_INVALID_ARG;
     pa_alloc_stats st = {};
     st.num_blocks = a->num_blocks;
-    st.free_blocks = (int64_t)a->free_list.size();
+    st.free_blocks = a->free_count;
     std::vector<int32_t> filled(a->num_blocks, 0);
     for (const auto &kv : a->seqs) {
         const Sequence &s = kv.second;
@@ -206,6 +262,9 @@ int pa_alloc_get_stats(const pa_alloc *a, pa_alloc_stats *out) {
         st.filled_slots += filled[b];
     }
     st.cow_copies = a->cow_copies;
+    st.cached_blocks = (int64_t)a->cached.size();
+    st.prefix_query_blocks = a->prefix_query_blocks;
+    st.prefix_hit_blocks = a->prefix_hit_blocks;
     st.usage = (double)st.used_blocks / (double)st.num_blocks;
     st.waste = st.used_blocks
                    ? 1.0 - (double)st.filled_slots / ((double)st.used_blocks * a->block_size)
@@ -213,6 +272,82 @@ int pa_alloc_get_stats(const pa_alloc *a, pa_alloc_stats *out) {
     st.sharing_saving =
         st.logical_blocks ? 1.0 - (double)st.used_blocks / (double)st.logical_blocks : 0.0;
     *out = st;
+    return PA_OK;
+}
+
+int pa_alloc_enable_prefix_caching(pa_alloc *a, int32_t enable) {
+    if (!a) return PA_ERR_INVALID_ARG;
+    if (enable && a->block_tokens.empty())
+        a->block_tokens.assign((size_t)a->num_blocks * a->block_size, 0);
+    if (!enable) {
+        for (int32_t b = 0; b < a->num_blocks; ++b) a->unregister(b);
+    }
+    a->prefix_caching = enable != 0;
+    return PA_OK;
+}
+
+int pa_alloc_add_seq_tokens(pa_alloc *a, int64_t seq_id, const int32_t *tokens,
+                            int32_t num_tokens, int32_t *num_cached_tokens) {
+    if (!a || num_tokens < 0 || (num_tokens > 0 && !tokens) || !num_cached_tokens ||
+        a->seqs.count(seq_id))
+        return PA_ERR_INVALID_ARG;
+    const int32_t bs = a->block_size;
+    const int64_t need = a->blocks_for(num_tokens);
+    const int32_t full = num_tokens / bs;
+    // 1. leading full blocks already in the cache (chain hash + exact tokens)
+    std::vector<uint64_t> hashes(full);
+    std::vector<int32_t> hits;
+    uint64_t h = kFnvOffset;
+    for (int32_t i = 0; i < full; ++i) {
+        h = fnv1a(h, tokens + (size_t)i * bs, sizeof(int32_t) * bs);
+        hashes[i] = h;
+    }
+    if (a->prefix_caching) {
+        for (int32_t i = 0; i < full; ++i) {
+            auto it = a->cached.find(hashes[i]);
+            if (it == a->cached.end()) break;
+            const int32_t b = it->second;
+            if (std::memcmp(&a->block_tokens[(size_t)b * bs], tokens + (size_t)i * bs,
+                            sizeof(int32_t) * bs) != 0)
+                break;
+            hits.push_back(b);
+        }
+    }
+    // 2. enough free blocks for the rest?  (a hit that sits on the free list
+    // leaves it, so it cannot also be claimed)
+    int64_t hits_on_free = 0;
+    for (int32_t b : hits) hits_on_free += a->in_free[b];
+    if (need - (int64_t)hits.size() > a->free_count - hits_on_free) return PA_ERR_NO_BLOCKS;
+    // 3. commit
+    Sequence s;
+    s.num_tokens = num_tokens;
+    s.blocks.reserve(need);
+    for (int32_t b : hits) {
+        if (a->in_free[b]) {
+            a->unlink_free(b);
+            a->refcount[b] = 1;
+        } else {
+            ++a->refcount[b];
+        }
+        s.blocks.push_back(b);
+    }
+    for (int64_t i = (int64_t)hits.size(); i < need; ++i) {
+        const int32_t b = a->claim();
+        s.blocks.push_back(b);
+        if (a->prefix_caching && i < full && !a->cached.count(hashes[i])) {
+            a->cached.emplace(hashes[i], b);
+            a->block_hash[b] = hashes[i];
+            a->registered[b] = 1;
+            std::memcpy(&a->block_tokens[(size_t)b * bs], tokens + (size_t)i * bs,
+                        sizeof(int32_t) * bs);
+        }
+    }
+    if (a->prefix_caching) {
+        a->prefix_query_blocks += full;
+        a->prefix_hit_blocks += (int64_t)hits.size();
+    }
+    *num_cached_tokens = (int32_t)hits.size() * bs;
+    a->seqs.emplace(seq_id, std::move(s));
     return PA_OK;
 }
 

@@ -247,3 +247,135 @@ def test_pool_budget_reproduces_printed_figure():
     assert pk.pool_bytes(8e9, 16e9, 0.9) == 0.0
     blocks = pk.pool_num_blocks(got * 1e9, 32, 8, 128, 16, 2)  # Llama-3.1-8B shape
     assert blocks == int(7.2e9 // (16 * 2 * 32 * 8 * 128 * 2))
+
+
+# ---------------------------------------------------------------- automatic prefix caching
+def _tokens(rng, n):
+    return rng.integers(0, 32000, size=n).astype(np.int32)
+
+
+def test_prefix_cache_shares_matching_full_blocks():
+    rng = np.random.default_rng(3)
+    a = pk.BlockAllocator(32)
+    a.enable_prefix_caching()
+    system = _tokens(rng, 40)                       # 2 full blocks + 8 tokens
+    p1 = np.concatenate([system, _tokens(rng, 5)])
+    p2 = np.concatenate([system, _tokens(rng, 30)])
+    assert a.add_seq_tokens(1, p1) == 0
+    assert a.add_seq_tokens(2, p2) == 32            # the two full blocks are reused
+    t1, t2 = a.block_table(1), a.block_table(2)
+    assert list(t1[:2]) == list(t2[:2]) and t1[2] != t2[2]
+    assert [a.refcount(b) for b in t1[:2]] == [2, 2]
+    st = a.stats()
+    assert st["prefix_hit_blocks"] == 2 and st["prefix_query_blocks"] == 2 + 4
+    assert st["cached_blocks"] == 2 + 2             # p2's own third and fourth full blocks
+
+
+def test_prefix_cache_matches_only_whole_prefixes():
+    rng = np.random.default_rng(4)
+    a = pk.BlockAllocator(32)
+    a.enable_prefix_caching()
+    base = _tokens(rng, 48)
+    a.add_seq_tokens(1, base)
+    other = base.copy()
+    other[20] += 1                                  # differs inside block 1
+    assert a.add_seq_tokens(2, other) == 16          # only block 0 matches
+    shifted = np.concatenate([_tokens(rng, 16), base[16:32]])
+    assert a.add_seq_tokens(3, shifted) == 0         # same block content, other prefix
+    assert a.add_seq_tokens(4, base[:47]) == 32      # partial last block is never shared
+
+
+def test_freed_cached_blocks_stay_findable_until_reused():
+    rng = np.random.default_rng(5)
+    a = pk.BlockAllocator(6)
+    a.enable_prefix_caching()
+    p = _tokens(rng, 48)                            # 3 full blocks
+    a.add_seq_tokens(1, p)
+    a.free_seq(1)
+    assert a.stats()["free_blocks"] == 6 and a.stats()["cached_blocks"] == 3
+    assert a.add_seq_tokens(2, p) == 48             # revived from the free list
+    assert a.stats()["free_blocks"] == 3
+    a.free_seq(2)
+    a.add_seq(3, 16 * 4)                            # 4 blocks: 3 never-used, then evicts one
+    assert a.stats()["cached_blocks"] == 2
+    a.free_seq(3)
+    assert a.add_seq_tokens(4, p) == 0              # the first cached block was evicted
+
+
+def test_prefix_cache_off_behaves_like_add_seq():
+    rng = np.random.default_rng(6)
+    a = pk.BlockAllocator(8)
+    p = _tokens(rng, 40)
+    assert a.add_seq_tokens(1, p) == 0
+    assert a.add_seq_tokens(2, p) == 0
+    assert list(a.block_table(1)) == [0, 1, 2] and list(a.block_table(2)) == [3, 4, 5]
+    assert a.stats()["cached_blocks"] == 0
+
+
+def test_prefix_cache_exhaustion_leaves_state_unchanged():
+    rng = np.random.default_rng(7)
+    a = pk.BlockAllocator(5)
+    a.enable_prefix_caching()
+    p = _tokens(rng, 32)
+    a.add_seq_tokens(1, p)                          # 2 blocks
+    a.add_seq(2, 48)                                # 3 blocks: pool full
+    before = a.stats()
+    with pytest.raises(pk.PagedError) as e:
+        a.add_seq_tokens(3, np.concatenate([p, _tokens(rng, 1)]))  # 2 hits + 1 new: none free
+    assert e.value.status == pk.PA_ERR_NO_BLOCKS and a.stats() == before
+    a.free_seq(2)
+    assert a.add_seq_tokens(3, np.concatenate([p, _tokens(rng, 1)])) == 32
+
+
+def test_prefix_cache_hit_rate_on_shared_system_prompt():
+    """Requests that share a 512-token system prompt reuse its 32 blocks:
+    every request after the first hits all of them."""
+    rng = np.random.default_rng(8)
+    a = pk.BlockAllocator(4096)
+    a.enable_prefix_caching()
+    system = _tokens(rng, 512)
+    for r in range(50):
+        user = _tokens(rng, int(rng.integers(1, 300)))
+        cached = a.add_seq_tokens(r, np.concatenate([system, user]))
+        assert cached >= (0 if r == 0 else 512)
+    st = a.stats()
+    assert st["prefix_hit_blocks"] == 49 * 32
+    assert st["prefix_hit_blocks"] / st["prefix_query_blocks"] > 0.5
+
+
+def test_random_operations_with_prefix_cache_keep_the_pool_consistent():
+    rng = np.random.default_rng(9)
+    a = pk.BlockAllocator(120)
+    a.enable_prefix_caching()
+    prompts = [_tokens(rng, int(rng.integers(1, 80))) for _ in range(6)]
+    live, next_id = set(), 0
+    for _ in range(2000):
+        op = rng.integers(0, 4)
+        try:
+            if op == 0 or not live:
+                base = prompts[int(rng.integers(0, 6))]
+                p = np.concatenate([base, _tokens(rng, int(rng.integers(0, 20)))])
+                cached = a.add_seq_tokens(next_id, p)
+                assert cached % 16 == 0 and cached <= len(p)
+                live.add(next_id)
+                next_id += 1
+            elif op == 1:
+                a.append_slot(int(rng.choice(sorted(live))))
+            elif op == 2:
+                s = int(rng.choice(sorted(live)))
+                a.fork(s, next_id)
+                live.add(next_id)
+                next_id += 1
+            else:
+                s = int(rng.choice(sorted(live)))
+                a.free_seq(s)
+                live.discard(s)
+        except pk.PagedError as e:
+            assert e.status == pk.PA_ERR_NO_BLOCKS
+        holders = np.zeros(120, np.int64)
+        for s in live:
+            np.add.at(holders, a.block_table(s), 1)
+        rc = np.array([a.refcount(b) for b in range(120)])
+        assert np.array_equal(rc, holders)
+        st = a.stats()
+        assert st["free_blocks"] + st["used_blocks"] == 120

@@ -289,3 +289,51 @@ def test_host_side_rejections():
         kc3 = torch.zeros((4, 3, 16, 64), dtype=torch.float16, device="cuda")
         pk.decode(q.clone(), q, kc3, kc3, tb[:, :2].contiguous(), ln, 3, 0.1)
     assert e.value.status == pk.PA_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- automatic prefix caching
+def test_prefix_cached_requests_decode_like_unshared_ones():
+    """Requests sharing a 96-token system prompt: the allocator reuses its 6
+    cached blocks, K/V are written only for the tokens after them, and every
+    request's decode equals attention over its own dense rows."""
+    import torch.nn.functional as F
+    rng = wl.rng_for(19)
+    H, Hq, d, dt, nb = 4, 8, 128, wl.BF16, 200
+    a = pk.BlockAllocator(nb)
+    a.enable_prefix_caching()
+    system = rng.integers(0, 32000, 96).astype(np.int32)
+    sys_k = wl.draw_values(rng, (96, H, d), dt)
+    sys_v = wl.draw_values(rng, (96, H, d), dt)
+    kc = wl.draw_values(rng, (nb, H, 16, d), dt)
+    vc = wl.draw_values(rng, (nb, H, 16, d), dt)
+    dkc, dvc = gh.to_dev(kc, dt), gh.to_dev(vc, dt)
+    dense_k, dense_v = [], []
+    for r in range(5):
+        n_user = int(rng.integers(1, 100))
+        toks = np.concatenate([system, rng.integers(0, 32000, n_user).astype(np.int32)])
+        k_rows = np.concatenate([sys_k, wl.draw_values(rng, (n_user, H, d), dt)])
+        v_rows = np.concatenate([sys_v, wl.draw_values(rng, (n_user, H, d), dt)])
+        cached = a.add_seq_tokens(r, toks)
+        assert cached == (0 if r == 0 else 96)
+        t = a.block_table(r)
+        pos = np.arange(cached, len(toks))
+        slots = (t[pos // 16].astype(np.int64) * 16 + pos % 16)
+        pk.reshape_and_cache(gh.to_dev(k_rows[cached:], dt), gh.to_dev(v_rows[cached:], dt), dkc,
+                             dvc, gh.ints(slots, torch.int64))
+        oracle.reshape_and_cache(k_rows[cached:], v_rows[cached:], kc, vc, slots)
+        dense_k.append(k_rows)
+        dense_v.append(v_rows)
+    tables, lens = a.build_tables(np.arange(5), 16)
+    q = wl.draw_values(rng, (5, Hq, d), dt)
+    out = gh.run_decode(pk, q, dkc, dvc, tables, lens, H, 1 / np.sqrt(d), dt)
+    assert pk.get_error() == (0, 0)
+    assert np.array_equal(gh.to_host_bits(dkc), kc)
+    ref = oracle.decode(q, kc, vc, tables, lens, H, 1 / np.sqrt(d), dt)
+    assert gh.max_err(out, ref) <= gh.TOL[dt]
+    for r in range(5):
+        qq = torch.from_numpy(bits_f64(q[r], dt)).reshape(1, Hq, 1, d)
+        kk = torch.from_numpy(bits_f64(dense_k[r], dt)).permute(1, 0, 2).unsqueeze(0)
+        vv = torch.from_numpy(bits_f64(dense_v[r], dt)).permute(1, 0, 2).unsqueeze(0)
+        dense = F.scaled_dot_product_attention(qq, kk, vv, scale=1 / np.sqrt(d), enable_gqa=True)
+        assert gh.max_err(out[r], dense.reshape(Hq, d).numpy()) <= gh.TOL[dt]
+    assert a.stats()["prefix_hit_blocks"] == 4 * 6
