@@ -49,7 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b",
-                    choices=["llama7b", "llama13b", "gqa_long", "cow", "tiny"])
+                    choices=["llama7b", "llama13b", "gqa_long", "cow", "tiny", "swap"])
     ap.add_argument("--layers", type=int, default=0,
                     help="layer caches to allocate (0: the workload's layer count; fewer "
                          "caches are cycled so every step still runs every layer)")
@@ -272,6 +272,8 @@ class Setup:
         self.parts = (b.max_blocks + 31) // 32
         self.stream = torch.cuda.current_stream(device)
         self.bytes_per_call = algorithmic_bytes(b.context_lens, Hq, H, d)
+        # K/V bytes of distinct physical blocks (shared prompt blocks once)
+        self.unique_kv_bytes = int(b.alloc.stats()["filled_slots"]) * H * d * 2 * 2
         self.launches_per_step = L * (1 + 1 + (1 if self.parts > 1 else 0)
                                       + (1 if self.pairs is not None else 0))
 
@@ -370,6 +372,7 @@ def run_ours(args, world, rank, local):
         "config": {**describe(st.w, st.batch.context_lens, st.ncache), "parallelism": f"replicas x{world}",
                    "num_blocks": st.nb, "decode_partitions": st.parts,
                    "cow_pairs_per_layer": 0 if st.pairs is None else int(st.pairs.shape[0]),
+                   "unique_kv_bytes_per_call": st.unique_kv_bytes,
                    "host_alloc_seconds": round(st.alloc_seconds, 3)},
         "kv_gbs": round(achieved, 1),
         "hbm_frac": round(achieved / peak, 4),
@@ -530,9 +533,57 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_swap(args):
+    """Swap bandwidth: scattered blocks of the Llama-7B layer shape (32 kv
+    heads x 16 x 128, fp16; 128 KiB per K or V block) between the device
+    pool and a pinned host pool, through pa_swap_blocks."""
+    import torch
+    import paged_kv_cache_425_b200 as pk
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nb_dev, nb_host, n = 8192, 4096, 2048
+    shape = (32, 16, 128)
+    kc = torch.randn((nb_dev, *shape), device=dev, dtype=torch.float16)
+    vc = torch.randn_like(kc)
+    hk = torch.empty((nb_host, *shape), dtype=torch.float16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    rng = wl.rng_for(args.seed)
+    src = rng.choice(nb_dev, n, replace=False).astype(np.int32)
+    dst = rng.choice(nb_host, n, replace=False).astype(np.int32)
+    out_pairs = np.stack([src, dst], axis=1)
+    in_pairs = np.stack([dst, rng.choice(nb_dev, n, replace=False).astype(np.int32)], axis=1)
+    bytes_each = 2 * n * 32 * 16 * 128 * 2
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    ms_out = timed(lambda: pk.swap_blocks(kc, vc, hk, hv, out_pairs))
+    ms_in = timed(lambda: pk.swap_blocks(hk, hv, kc, vc, in_pairs))
+    print(json.dumps({
+        "metric": "block swap bandwidth (device <-> pinned host)", "value": round(bytes_each / (ms_in * 1e-3) / 1e9, 2),
+        "unit": "GB/s (swap in)", "swap_out_gbs": round(bytes_each / (ms_out * 1e-3) / 1e9, 2),
+        "bytes_per_direction": bytes_each, "blocks": n, "block_bytes_k_or_v": 32 * 16 * 128 * 2,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": "f16",
+        "config": {"workload": "swap: 2048 scattered Llama-7B-shaped blocks, K and V"}}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_env()
+    if args.workload == "swap":
+        if rank == 0:
+            run_swap(args)
+        return 0
     if world > 1 and args.gpus != world:
         args.gpus = world
     if args.impl == "reference":

@@ -17,7 +17,12 @@
  *    matches reuses the cached physical blocks instead of recomputing them.
  *  - same page, section "Python LLM Inference Optimization with vLLM:
  *    Parameters That Actually Matter": the block pool takes a fraction
- *    (gpu_memory_utilization) of the memory left after the weights.
+ *    (gpu_memory_utilization) of the memory left after the weights; under
+ *    memory pressure sequences are swapped out or recomputed.
+ *  - "PagedAttention in vLLM: a throughput settings guide", section
+ *    "Continuous Batching Keeps the GPU Busy": the scheduler revisits the
+ *    batch every step, and too many sequences for the KV budget cause
+ *    preemption.
  *  - "vLLM PagedAttention: reducing KV cache memory waste", section "How
  *    PagedAttention Works": only a sequence's last block can be partly
  *    empty, so waste is bounded by one block per sequence.
@@ -138,6 +143,36 @@ int pa_alloc_add_seq_tokens(pa_alloc *a, int64_t seq_id, const int32_t *tokens,
 int32_t pa_alloc_refcount(const pa_alloc *a, int32_t block);
 
 int pa_alloc_get_stats(const pa_alloc *a, pa_alloc_stats *out);
+
+/* Result of pa_sim_continuous_batching. */
+typedef struct {
+    int64_t steps;            /* decoding steps simulated */
+    int64_t tokens_generated; /* new tokens produced (each counted once) */
+    int64_t preemptions;      /* sequences evicted for lack of blocks */
+    int64_t admitted;         /* admissions, re-admissions after preemption included */
+    int64_t finished;         /* requests that produced all their tokens */
+    int64_t rejected;         /* requests that could never fit in the pool */
+    double mean_usage;        /* mean fraction of pool blocks in use after a step */
+    double max_usage;
+    double mean_running;      /* mean sequences running after a step */
+} pa_sim_stats;
+
+/* Iteration-level scheduling ("continuous batching") on a pool of
+ * num_blocks blocks.  Request r has prompt_lens[r] prompt tokens and wants
+ * output_lens[r] >= 1 new tokens; all requests wait in a first-in-first-out
+ * queue at step 0.  Every step: (1) while fewer than max_num_seqs run, the
+ * queue's head is admitted if the pool can hold its prompt plus the tokens
+ * it generated before any preemption (that prefix is recomputed); (2) every
+ * running sequence appends one token; if the pool is out of blocks, the
+ * latest-admitted running sequence is preempted (its blocks freed at once,
+ * it returns to the front of the queue), repeatedly, until the append fits
+ * or the sequence itself was preempted; a sequence that produced all its
+ * tokens frees its blocks at once.  Requests whose whole life exceeds the
+ * pool are rejected up front.  Stops when every request finished or after
+ * max_steps. */
+int pa_sim_continuous_batching(int32_t num_blocks, int32_t block_size, int32_t max_num_seqs,
+                               const int32_t *prompt_lens, const int32_t *output_lens,
+                               int32_t num_requests, int64_t max_steps, pa_sim_stats *out);
 
 /* KV bytes one token occupies across all layers: 2 x layers x kv_heads x
  * head_dim x dtype_bytes (K and V). */

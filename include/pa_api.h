@@ -217,6 +217,34 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pa
                    int64_t num_blocks, int32_t dtype, void *stream);
 
 /*
+ * pa_swap_blocks - move whole blocks between two caches, one of which may
+ * live in page-locked host memory (swap out under memory pressure, swap back
+ * in later).
+ *
+ * Source: "Inside vLLM ...", section "Python LLM Inference Optimization with
+ * vLLM: Parameters That Actually Matter" (under memory pressure a sequence's
+ * blocks can be swapped to CPU RAM; swapping keeps the KV cache but costs
+ * PCIe bandwidth).
+ *
+ * For each pair p, block src_dst_pairs[p][1] of (dst_key_cache,
+ * dst_value_cache) becomes a bit-exact copy of block src_dst_pairs[p][0] of
+ * (src_key_cache, src_value_cache).  Both caches have the layout above with
+ * the same num_kv_heads, head_dim and dtype; each may be device memory or
+ * page-locked host memory (pageable host memory works but the copy is not
+ * asynchronous).  The pairs are a HOST array: the copies are issued from the
+ * host as one cudaMemcpyAsync per run of consecutive source and destination
+ * ids, K and V separately.  An id out of range returns PA_ERR_OUT_OF_RANGE
+ * before anything is enqueued.  Destinations must be distinct and must not
+ * be sources of the same call when both caches are the same memory.
+ *
+ *   src_dst_pairs  host, int32 [num_pairs][2]
+ */
+int pa_swap_blocks(const void *src_key_cache, const void *src_value_cache, int64_t src_num_blocks,
+                   void *dst_key_cache, void *dst_value_cache, int64_t dst_num_blocks,
+                   const int32_t *src_dst_pairs, int32_t num_pairs, int32_t num_kv_heads,
+                   int32_t head_dim, int32_t block_size, int32_t dtype, void *stream);
+
+/*
  * pa_get_error - synchronise `stream`, then read and clear the device error
  * word (one word for the whole process and device).  *bits (host, may be
  * NULL) receives the PA_DEVERR_* bits seen since the last call.  Returns

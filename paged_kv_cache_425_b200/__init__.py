@@ -57,6 +57,12 @@ def _sig(name, restype, *argtypes):
     return fn
 
 
+class SimStats(ctypes.Structure):
+    _fields_ = [("steps", _i64), ("tokens_generated", _i64), ("preemptions", _i64),
+                ("admitted", _i64), ("finished", _i64), ("rejected", _i64),
+                ("mean_usage", _f64), ("max_usage", _f64), ("mean_running", _f64)]
+
+
 class AllocStats(ctypes.Structure):
     _fields_ = [("num_blocks", _i64), ("free_blocks", _i64), ("used_blocks", _i64),
                 ("shared_blocks", _i64), ("num_seqs", _i64), ("logical_tokens", _i64),
@@ -75,6 +81,8 @@ pa_decode_static_workspace = _sig("pa_decode_static_workspace", ctypes.c_int, _P
                                   _P, _i32, _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
 pa_copy_blocks = _sig("pa_copy_blocks", ctypes.c_int, _P, _P, _P, _i32, _i32, _i32, _i32, _i64,
                       _i32, _P)
+pa_swap_blocks = _sig("pa_swap_blocks", ctypes.c_int, _P, _P, _i64, _P, _P, _i64, _P, _i32, _i32,
+                      _i32, _i32, _i32, _P)
 pa_get_error = _sig("pa_get_error", ctypes.c_int, _P, ctypes.POINTER(ctypes.c_uint32))
 pa_status_string = _sig("pa_status_string", ctypes.c_char_p, ctypes.c_int)
 pa_version = _sig("pa_version", ctypes.c_int)
@@ -95,6 +103,8 @@ pa_alloc_enable_prefix_caching = _sig("pa_alloc_enable_prefix_caching", ctypes.c
 pa_alloc_add_seq_tokens = _sig("pa_alloc_add_seq_tokens", ctypes.c_int, _P, _i64, _P, _i32,
                                ctypes.POINTER(_i32))
 pa_alloc_get_stats = _sig("pa_alloc_get_stats", ctypes.c_int, _P, ctypes.POINTER(AllocStats))
+pa_sim_continuous_batching = _sig("pa_sim_continuous_batching", ctypes.c_int, _i32, _i32, _i32,
+                                  _P, _P, _i32, _i64, ctypes.POINTER(SimStats))
 pa_kv_bytes_per_token = _sig("pa_kv_bytes_per_token", _i64, _i32, _i32, _i32, _i32)
 pa_pool_bytes = _sig("pa_pool_bytes", _f64, _f64, _f64, _f64)
 pa_pool_num_blocks = _sig("pa_pool_num_blocks", _i64, _f64, _i32, _i32, _i32, _i32, _i32)
@@ -233,6 +243,27 @@ def copy_blocks(key_cache, value_cache, src_dst_pairs, stream=None):
                           hkv, d, bs, nb, dtype_code(key_cache), _stream(stream)), "pa_copy_blocks")
 
 
+def swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, src_dst_pairs,
+                stream=None):
+    """Copy whole blocks between two caches (device or pinned host tensors);
+    src_dst_pairs is a host int32 array [P][2]."""
+    snb, hkv, bs, d = _cache_shape(src_key_cache, src_value_cache)
+    dnb, hkv2, bs2, d2 = _cache_shape(dst_key_cache, dst_value_cache)
+    if (hkv, bs, d) != (hkv2, bs2, d2) or src_key_cache.dtype != dst_key_cache.dtype:
+        raise ValueError("source and destination caches must have the same block shape")
+    for t, n in ((src_key_cache, "src_key_cache"), (src_value_cache, "src_value_cache"),
+                 (dst_key_cache, "dst_key_cache"), (dst_value_cache, "dst_value_cache")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    pairs = np.ascontiguousarray(src_dst_pairs, dtype=np.int32).reshape(-1, 2)
+    _check(pa_swap_blocks(ctypes.c_void_p(src_key_cache.data_ptr()),
+                          ctypes.c_void_p(src_value_cache.data_ptr()), snb,
+                          ctypes.c_void_p(dst_key_cache.data_ptr()),
+                          ctypes.c_void_p(dst_value_cache.data_ptr()), dnb,
+                          pairs.ctypes.data if len(pairs) else None, int(len(pairs)), hkv, d, bs,
+                          dtype_code(src_key_cache), _stream(stream)), "pa_swap_blocks")
+
+
 def get_error(stream=None):
     """Synchronise the stream, return (status, PA_DEVERR_* bits) and clear them."""
     bits = ctypes.c_uint32(0)
@@ -326,6 +357,19 @@ class BlockAllocator:
         st = AllocStats()
         _check(pa_alloc_get_stats(self._h, ctypes.byref(st)), "pa_alloc_get_stats")
         return {name: getattr(st, name) for name, _ in AllocStats._fields_}
+
+
+def simulate_continuous_batching(num_blocks: int, max_num_seqs: int, prompt_lens, output_lens,
+                                 block_size: int = BLOCK_SIZE, max_steps: int = 10_000_000) -> dict:
+    """Iteration-level scheduling over the allocator; returns the stats dict."""
+    pl = np.ascontiguousarray(prompt_lens, dtype=np.int32)
+    ol = np.ascontiguousarray(output_lens, dtype=np.int32)
+    st = SimStats()
+    _check(pa_sim_continuous_batching(num_blocks, block_size, max_num_seqs,
+                                      pl.ctypes.data if pl.size else None,
+                                      ol.ctypes.data if ol.size else None, int(pl.size),
+                                      max_steps, ctypes.byref(st)), "pa_sim_continuous_batching")
+    return {name: getattr(st, name) for name, _ in SimStats._fields_}
 
 
 def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, dtype_bytes: int) -> int:

@@ -22,7 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("pa_api.cu", "pa_alloc.cc")]
+SOURCES = [os.path.join(CSRC, f) for f in ("pa_api.cu", "pa_alloc.cc", "pa_sim.cc")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_device.cuh")] + [
     os.path.join(INCLUDE, f) for f in ("pa_api.h", "pa_alloc.h")]
 

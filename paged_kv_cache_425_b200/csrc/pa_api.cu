@@ -279,6 +279,46 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pa
                       vec_per_block);
 }
 
+int pa_swap_blocks(const void *src_key_cache, const void *src_value_cache, int64_t src_num_blocks,
+                   void *dst_key_cache, void *dst_value_cache, int64_t dst_num_blocks,
+                   const int32_t *src_dst_pairs, int32_t num_pairs, int32_t num_kv_heads,
+                   int32_t head_dim, int32_t block_size, int32_t dtype, void *stream) {
+    int rc = check_cache_shape(num_kv_heads, head_dim, block_size,
+                               src_num_blocks > dst_num_blocks ? src_num_blocks : dst_num_blocks,
+                               dtype);
+    if (rc != PA_OK) return rc;
+    if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!src_key_cache || !src_value_cache || !dst_key_cache || !dst_value_cache ||
+        !src_dst_pairs)
+        return PA_ERR_INVALID_ARG;
+    for (int32_t p = 0; p < num_pairs; ++p) {
+        const int64_t s = src_dst_pairs[2 * p], d = src_dst_pairs[2 * p + 1];
+        if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) return PA_ERR_OUT_OF_RANGE;
+    }
+    const size_t block_bytes = (size_t)num_kv_heads * kBlock * head_dim * 2;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const char *sk = static_cast<const char *>(src_key_cache);
+    const char *sv = static_cast<const char *>(src_value_cache);
+    char *dk = static_cast<char *>(dst_key_cache);
+    char *dv = static_cast<char *>(dst_value_cache);
+    for (int32_t p = 0; p < num_pairs;) {
+        // extend a run while both ids advance by one
+        int32_t q = p + 1;
+        while (q < num_pairs && src_dst_pairs[2 * q] == src_dst_pairs[2 * (q - 1)] + 1 &&
+               src_dst_pairs[2 * q + 1] == src_dst_pairs[2 * (q - 1) + 1] + 1)
+            ++q;
+        const size_t off_s = (size_t)src_dst_pairs[2 * p] * block_bytes;
+        const size_t off_d = (size_t)src_dst_pairs[2 * p + 1] * block_bytes;
+        const size_t n = (size_t)(q - p) * block_bytes;
+        if (cudaMemcpyAsync(dk + off_d, sk + off_s, n, cudaMemcpyDefault, st) != cudaSuccess ||
+            cudaMemcpyAsync(dv + off_d, sv + off_s, n, cudaMemcpyDefault, st) != cudaSuccess)
+            return PA_ERR_CUDA;
+        p = q;
+    }
+    return PA_OK;
+}
+
 int pa_get_error(void *stream, uint32_t *bits) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;

@@ -379,3 +379,58 @@ def test_random_operations_with_prefix_cache_keep_the_pool_consistent():
         assert np.array_equal(rc, holders)
         st = a.stats()
         assert st["free_blocks"] + st["used_blocks"] == 120
+
+
+def test_swap_rejects_bad_ids_before_any_copy():
+    """Host-side check: no CUDA call happens for an out-of-range pair."""
+    buf = np.zeros(4 * 2 * 16 * 64, np.uint16)
+    pairs = np.array([[0, 1], [5, 2]], np.int32)  # source 5 of a 4-block pool
+    rc = pk.pa_swap_blocks(buf.ctypes.data, buf.ctypes.data, 4, buf.ctypes.data, buf.ctypes.data,
+                           4, pairs.ctypes.data, 2, 2, 64, 16, pk.F16, None)
+    assert rc == pk.PA_ERR_OUT_OF_RANGE
+    assert pk.pa_swap_blocks(buf.ctypes.data, buf.ctypes.data, 4, buf.ctypes.data,
+                             buf.ctypes.data, 4, pairs.ctypes.data, 2, 2, 96, 16, pk.F16,
+                             None) == pk.PA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- continuous batching simulation
+def _requests(seed=0, n=200):
+    rng = np.random.default_rng(seed)
+    return rng.integers(50, 500, n).astype(np.int32), rng.integers(1, 300, n).astype(np.int32)
+
+
+def test_simulation_finishes_everything_and_counts_each_token_once():
+    pl, ol = _requests()
+    for nb, m in ((20000, 64), (600, 64), (300, 256)):
+        st = pk.simulate_continuous_batching(nb, m, pl, ol)
+        assert st["finished"] == len(pl) and st["rejected"] == 0
+        assert st["tokens_generated"] == int(ol.sum())
+        assert st["admitted"] == len(pl) + st["preemptions"]
+        assert 0 < st["mean_usage"] <= st["max_usage"] <= 1.0
+
+
+def test_ample_pool_never_preempts_and_one_slot_is_sequential():
+    pl, ol = _requests(1, 50)
+    assert pk.simulate_continuous_batching(100000, 64, pl, ol)["preemptions"] == 0
+    st = pk.simulate_continuous_batching(100000, 1, pl, ol)
+    assert st["steps"] == int(ol.sum()) and st["mean_running"] <= 1.0
+
+
+def test_too_few_sequences_starve_and_too_many_preempt():
+    """'PagedAttention in vLLM: a throughput settings guide', 'Continuous
+    Batching Keeps the GPU Busy': too low a max_num_seqs starves the GPU
+    (more steps for the same tokens), too high with a fixed KV budget
+    increases preemption."""
+    pl, ol = _requests(2)
+    low = pk.simulate_continuous_batching(600, 4, pl, ol)
+    mid = pk.simulate_continuous_batching(600, 16, pl, ol)
+    high = pk.simulate_continuous_batching(600, 256, pl, ol)
+    assert low["steps"] > mid["steps"]
+    assert low["preemptions"] == 0 and high["preemptions"] > mid["preemptions"]
+    assert high["max_usage"] == 1.0
+
+
+def test_requests_larger_than_the_pool_are_rejected():
+    st = pk.simulate_continuous_batching(10, 4, np.array([100, 400], np.int32),
+                                         np.array([10, 10], np.int32))
+    assert st["rejected"] == 1 and st["finished"] == 1

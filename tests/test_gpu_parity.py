@@ -337,3 +337,40 @@ def test_prefix_cached_requests_decode_like_unshared_ones():
         dense = F.scaled_dot_product_attention(qq, kk, vv, scale=1 / np.sqrt(d), enable_gqa=True)
         assert gh.max_err(out[r], dense.reshape(Hq, d).numpy()) <= gh.TOL[dt]
     assert a.stats()["prefix_hit_blocks"] == 4 * 6
+
+
+# ---------------------------------------------------------------- swap out / swap in
+def test_swap_out_and_back_in_is_bit_exact_and_decode_follows():
+    """A sequence's blocks go to a pinned host pool and come back into other
+    device blocks; the bytes round-trip exactly and decode through the
+    remapped table gives the same bits as before."""
+    rng = wl.rng_for(20)
+    H, d, dt = 8, 128, wl.BF16
+    lens = np.array([300, 77], np.int32)
+    nb = 64
+    p = make_paged(rng, 2, 16, H, d, lens, nb, dt)
+    before = gh.to_host_bits(gpu_out(p))
+    dkc, dvc = gh.to_dev(p.key_cache, dt), gh.to_dev(p.value_cache, dt)
+    host_k = torch.zeros((40, H, 16, d), dtype=torch.bfloat16).pin_memory()
+    host_v = torch.zeros_like(host_k).pin_memory()
+    n0 = (int(lens[0]) + 15) // 16
+    out_pairs = np.stack([p.tables[0, :n0], 5 + np.arange(n0)], axis=1).astype(np.int32)
+    pk.swap_blocks(dkc, dvc, host_k, host_v, out_pairs)
+    torch.cuda.synchronize()
+    hk = host_k.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(hk[5:5 + n0], p.key_cache[p.tables[0, :n0]])
+    # back into device blocks no table uses (sequence 1 keeps its blocks)
+    used = set(p.tables[:, :].ravel().tolist())
+    free = np.array([b for b in range(nb) if b not in used][:n0] if nb - len(used) >= n0 else [], np.int32)
+    if len(free) < n0:  # reuse sequence 0's own old blocks in reverse order
+        free = p.tables[0, :n0][::-1].copy()
+    in_pairs = np.stack([5 + np.arange(n0), free], axis=1).astype(np.int32)
+    pk.swap_blocks(host_k, host_v, dkc, dvc, in_pairs)
+    torch.cuda.synchronize()
+    tables = p.tables.copy()
+    tables[0, :n0] = free
+    after = gh.to_host_bits(gh.run_decode(pk, p.q, dkc, dvc, tables, lens, H, p.scale, dt))
+    assert np.array_equal(before, after)
+    with pytest.raises(pk.PagedError) as e:
+        pk.swap_blocks(dkc, dvc, host_k, host_v, np.array([[0, 40]], np.int32))
+    assert e.value.status == pk.PA_ERR_OUT_OF_RANGE

@@ -69,7 +69,7 @@ WORKLOADS = {
     # Llama-3.1-8B GQA long context: 32 seqs, 32 q / 8 kv heads, bf16
     "gqa_long": Workload("gqa_long", 32, 32, 8, 128, 16, BF16, 32, ("uniform", 8192, 32768)),
     # parallel sampling: 32 prompts x 4 branches of a 1000-token prompt
-    "cow": Workload("cow", 128, 32, 32, 128, 16, BF16, 1, ("fixed", 1000), prompts=32, branches=4,
+    "cow": Workload("cow", 128, 32, 32, 128, 16, BF16, 32, ("fixed", 1000), prompts=32, branches=4,
                     prompt_len=1000, own_max=256),
 }
 
