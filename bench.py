@@ -132,7 +132,7 @@ def load_peak():
 def kernel_source_digest() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("pa_kernels.cuh", "pa_device.cuh", "pa_api.cu"):
+    for f in ("pa_kernels.cuh", "pa_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_425_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -230,11 +230,14 @@ int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pa
  * dst_value_cache) becomes a bit-exact copy of block src_dst_pairs[p][0] of
  * (src_key_cache, src_value_cache).  Both caches have the layout above with
  * the same num_kv_heads, head_dim and dtype; each may be device memory or
- * page-locked host memory (pageable host memory works but the copy is not
- * asynchronous).  The pairs are a HOST array: the copies are issued from the
- * host as one cudaMemcpyAsync per run of consecutive source and destination
- * ids, K and V separately.  An id out of range returns PA_ERR_OUT_OF_RANGE
- * before anything is enqueued.  Destinations must be distinct and must not
+ * page-locked host memory.  The pairs are a HOST array.  When every pool is
+ * device memory of the current device or mapped page-locked host memory, one
+ * kernel per 2048 pairs moves the blocks (host pools through their device
+ * alias, over PCIe / C2C); otherwise (pageable host memory, another device)
+ * the copies are one cudaMemcpyAsync per run of consecutive source and
+ * destination ids, K and V separately, and pageable memory makes them
+ * synchronous.  An id out of range returns PA_ERR_OUT_OF_RANGE before
+ * anything is enqueued.  Destinations must be distinct and must not
  * be sources of the same call when both caches are the same memory.
  *
  *   src_dst_pairs  host, int32 [num_pairs][2]

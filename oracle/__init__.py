@@ -11,9 +11,10 @@ first use and marshals numpy arrays into it.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against things
 other than itself: exhaustive fp16 / bf16 widening against numpy, torch's
-fp64 scaled-dot-product attention on densely stored K/V, closed forms
-(one token, identical keys, constant values, two-token logistic weights) and
-invariants (physical block placement, split-range merge).
+fp64 scaled-dot-product attention on densely stored K/V (with a causal mask
+for chunked prefill), closed forms (one token, identical keys, constant
+values, two-token logistic weights) and invariants (physical block
+placement, split-range merge, a one-token chunk equals decode).
 """
 from __future__ import annotations
 
@@ -67,6 +68,9 @@ def _load(path: str | None = None):
             lib.oracle_decode_range.restype = None
             lib.oracle_lse_merge.argtypes = [P, P, P, i64, i32, i32]
             lib.oracle_lse_merge.restype = None
+            lib.oracle_prefill.argtypes = [P, P, P, P, P, i32, P, P, i32, i32, i32, i32, i32, f64,
+                                           i32]
+            lib.oracle_prefill.restype = None
             if path is not None:
                 return lib
             _lib = lib
@@ -157,6 +161,27 @@ def decode(q, key_cache, value_cache, block_tables, context_lens, num_kv_heads: 
     """softmax(scale q K^T) V per (seq, q head) over the whole paged context, fp64."""
     return decode_range(q, key_cache, value_cache, block_tables, context_lens, num_kv_heads,
                         scale, dtype, 0, -1, seqs)[0]
+
+
+def prefill(q, key_cache, value_cache, block_tables, context_lens, query_start, num_kv_heads: int,
+            scale: float, dtype: int) -> np.ndarray:
+    """Chunked prefill: query rows query_start[s]..query_start[s+1]-1 are the
+    last tokens of sequence s and attend causally over its paged context.
+    q [T][Hq][d] bits -> out [T][Hq][d] float64."""
+    q = _req(q, np.uint16)
+    kc = _req(key_cache, np.uint16)
+    vc = _req(value_cache, np.uint16)
+    tables = _req(block_tables, np.int32)
+    lens = _req(context_lens, np.int32)
+    qs = _req(query_start, np.int32)
+    T, Hq, d = q.shape
+    nb, hkv, bs, d2 = kc.shape
+    assert d2 == d and hkv == num_kv_heads and Hq % hkv == 0 and qs[-1] == T
+    out = np.zeros((T, Hq, d), dtype=np.float64)
+    _load().oracle_prefill(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(tables),
+                           int(tables.shape[1]), _ptr(lens), _ptr(qs), int(lens.shape[0]), Hq, hkv,
+                           d, bs, float(scale), int(dtype))
+    return out
 
 
 def lse_merge(o_parts: np.ndarray, lse_parts: np.ndarray) -> np.ndarray:

@@ -20,6 +20,10 @@
  *  - "vLLM PagedAttention: reducing KV cache memory waste", section "How
  *    PagedAttention Works": blocks are claimed as tokens arrive; only a
  *    sequence's last block can be partly filled.
+ *  - "PagedAttention in vLLM: a throughput settings guide", section "Tuning
+ *    Batching, Prefill, and Cache": with chunked prefill a step fills its
+ *    token budget with chunks of prompts; a chunk's tokens attend to the
+ *    cached tokens before them and causally to each other.
  *
  * Cache layout (a reading; the pages fix none): key_cache and value_cache are
  * each [num_blocks][num_kv_heads][block_size][head_dim] of 16-bit elements,
@@ -223,6 +227,44 @@ void oracle_decode_range(double *out, double *lse, const uint16_t *q, const uint
         double r = attend(out + job * head_dim, qd, K, V, n, head_dim, scale);
         if (lse)
             lse[job] = r;
+        free(qd);
+        free(K);
+        free(V);
+    }
+}
+
+/* Chunked prefill over the paged cache.  Sequence s owns query rows
+ * query_start[s] .. query_start[s + 1] - 1 of q ([num_q_tokens][num_q_heads]
+ * [head_dim]); they are the last n_s = query_start[s + 1] - query_start[s]
+ * tokens of its context of L = context_lens[s] tokens, whose K/V are already
+ * in the cache.  Query row i of s sits at position p = L - n_s + i and
+ * attends to tokens 0 .. p (causal): out row = softmax(scale q K^T) V over
+ * those tokens, in double. */
+void oracle_prefill(double *out, const uint16_t *q, const uint16_t *key_cache,
+                    const uint16_t *value_cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens,
+                    const int32_t *query_start, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, double scale,
+                    int32_t dtype) {
+    int32_t group = num_q_heads / num_kv_heads;
+    int64_t rows = (int64_t)query_start[num_seqs] * num_q_heads;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t job = 0; job < rows; ++job) {
+        int32_t t = (int32_t)(job / num_q_heads);
+        int32_t h = (int32_t)(job % num_q_heads);
+        int32_t s = 0;
+        while (query_start[s + 1] <= t) ++s;
+        int32_t n_s = query_start[s + 1] - query_start[s];
+        int32_t pos = context_lens[s] - n_s + (t - query_start[s]);
+        int32_t n = pos + 1 > 0 ? pos + 1 : 0;
+        double *qd = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        double *K = (double *)malloc(sizeof(double) * (size_t)head_dim * (size_t)(n ? n : 1));
+        double *V = (double *)malloc(sizeof(double) * (size_t)head_dim * (size_t)(n ? n : 1));
+        for (int32_t i = 0; i < head_dim; ++i)
+            qd[i] = widen(q[((int64_t)t * num_q_heads + h) * head_dim + i], dtype);
+        gather(K, V, key_cache, value_cache, block_tables + (int64_t)s * max_blocks_per_seq, 0, n,
+               h / group, num_kv_heads, head_dim, block_size, dtype);
+        attend(out + job * head_dim, qd, K, V, n, head_dim, scale);
         free(qd);
         free(K);
         free(V);

@@ -143,6 +143,28 @@ int dispatch_decode(const DecodeArgs &a, int head_dim, int group, const CUtensor
                            : launch_decode<T, 64>(a, group, tmk, tmv, st);
 }
 
+// Device-side address of `p` on the current device: itself for device memory
+// of this device, the mapped alias for page-locked host memory.  False for
+// pageable host memory, another device's memory or a lookup failure.
+bool device_alias(const void *p, const void **out) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (attr.type == cudaMemoryTypeDevice && attr.device == dev && attr.devicePointer) {
+        *out = p;
+        return true;
+    }
+    if (attr.type == cudaMemoryTypeHost && attr.devicePointer) {
+        *out = attr.devicePointer;
+        return true;
+    }
+    return false;
+}
+
 int64_t num_parts_for(int32_t max_blocks_per_seq) {
     return (max_blocks_per_seq + kPartBlocks - 1) / kPartBlocks;
 }
@@ -298,6 +320,32 @@ int pa_swap_blocks(const void *src_key_cache, const void *src_value_cache, int64
     }
     const size_t block_bytes = (size_t)num_kv_heads * kBlock * head_dim * 2;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // One kernel over all pairs when every pool is device memory of this
+    // device or mapped page-locked host memory (reached through its device
+    // alias); otherwise one cudaMemcpyAsync per run of consecutive ids.
+    const void *alias[4];
+    const void *ptrs[4] = {src_key_cache, src_value_cache, dst_key_cache, dst_value_cache};
+    bool kernel_path = true;
+    for (int i = 0; i < 4 && kernel_path; ++i) kernel_path = device_alias(ptrs[i], &alias[i]);
+    if (kernel_path) {
+        const long long vec_per_block = (long long)block_bytes / 16;
+        const int threads = 256;
+        long long chunks = (vec_per_block + threads * 4 - 1) / (threads * 4);
+        if (chunks > 65535) chunks = 65535;
+        for (int32_t p0 = 0; p0 < num_pairs; p0 += kSwapChunk) {
+            const int n = num_pairs - p0 < kSwapChunk ? num_pairs - p0 : kSwapChunk;
+            SwapPairs pp;
+            for (int i = 0; i < n; ++i)
+                pp.p[i] = make_int2(src_dst_pairs[2 * (p0 + i)], src_dst_pairs[2 * (p0 + i) + 1]);
+            const int rc2 = launch_pdl(
+                swap_blocks_kernel, dim3(n, (unsigned)chunks), dim3(threads), 0, st,
+                static_cast<const uint4 *>(alias[0]), static_cast<const uint4 *>(alias[1]),
+                static_cast<uint4 *>(const_cast<void *>(alias[2])),
+                static_cast<uint4 *>(const_cast<void *>(alias[3])), pp, n, vec_per_block);
+            if (rc2 != PA_OK) return rc2;
+        }
+        return PA_OK;
+    }
     const char *sk = static_cast<const char *>(src_key_cache);
     const char *sv = static_cast<const char *>(src_value_cache);
     char *dk = static_cast<char *>(dst_key_cache);

@@ -720,4 +720,34 @@ __global__ void copy_blocks_kernel(uint4 *__restrict__ kc, uint4 *__restrict__ v
     }
 }
 
+// ------------------------------------------------------------------ block swap
+// Whole blocks between two pools, either of which may be mapped page-locked
+// host memory reached through its device alias: grid.x strides over pairs,
+// grid.y over 16-byte chunks of a block.  Ids were checked on the host.
+constexpr int kSwapChunk = 2048;  // pairs per launch, passed by value (16 KiB)
+struct SwapPairs {
+    int2 p[kSwapChunk];
+};
+
+__global__ void swap_blocks_kernel(const uint4 *__restrict__ sk, const uint4 *__restrict__ sv,
+                                   uint4 *__restrict__ dk, uint4 *__restrict__ dv,
+                                   const __grid_constant__ SwapPairs pairs, int num_pairs,
+                                   long long vec_per_block) {
+    pdl_launch_dependents();
+    pdl_wait_prior();
+    for (int p = blockIdx.x; p < num_pairs; p += gridDim.x) {
+        const int2 pr = pairs.p[p];
+        const uint4 *ks = sk + (long long)pr.x * vec_per_block;
+        const uint4 *vs = sv + (long long)pr.x * vec_per_block;
+        uint4 *kd = dk + (long long)pr.y * vec_per_block;
+        uint4 *vd = dv + (long long)pr.y * vec_per_block;
+        for (long long i = (long long)blockIdx.y * blockDim.x + threadIdx.x; i < vec_per_block;
+             i += (long long)gridDim.y * blockDim.x) {
+            const uint4 a = ks[i], b = vs[i];
+            kd[i] = a;
+            vd[i] = b;
+        }
+    }
+}
+
 }  // namespace pa

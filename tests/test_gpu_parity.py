@@ -340,10 +340,12 @@ def test_prefix_cached_requests_decode_like_unshared_ones():
 
 
 # ---------------------------------------------------------------- swap out / swap in
-def test_swap_out_and_back_in_is_bit_exact_and_decode_follows():
-    """A sequence's blocks go to a pinned host pool and come back into other
-    device blocks; the bytes round-trip exactly and decode through the
-    remapped table gives the same bits as before."""
+@pytest.mark.parametrize("pinned", [True, False], ids=["pinned-kernel", "pageable-copies"])
+def test_swap_out_and_back_in_is_bit_exact_and_decode_follows(pinned):
+    """A sequence's blocks go to a host pool and come back into other device
+    blocks; the bytes round-trip exactly and decode through the remapped
+    table gives the same bits as before.  A pinned pool takes the kernel
+    path, a pageable one the per-run copy path."""
     rng = wl.rng_for(20)
     H, d, dt = 8, 128, wl.BF16
     lens = np.array([300, 77], np.int32)
@@ -351,8 +353,10 @@ def test_swap_out_and_back_in_is_bit_exact_and_decode_follows():
     p = make_paged(rng, 2, 16, H, d, lens, nb, dt)
     before = gh.to_host_bits(gpu_out(p))
     dkc, dvc = gh.to_dev(p.key_cache, dt), gh.to_dev(p.value_cache, dt)
-    host_k = torch.zeros((40, H, 16, d), dtype=torch.bfloat16).pin_memory()
-    host_v = torch.zeros_like(host_k).pin_memory()
+    host_k = torch.zeros((40, H, 16, d), dtype=torch.bfloat16)
+    host_v = torch.zeros_like(host_k)
+    if pinned:
+        host_k, host_v = host_k.pin_memory(), host_v.pin_memory()
     n0 = (int(lens[0]) + 15) // 16
     out_pairs = np.stack([p.tables[0, :n0], 5 + np.arange(n0)], axis=1).astype(np.int32)
     pk.swap_blocks(dkc, dvc, host_k, host_v, out_pairs)

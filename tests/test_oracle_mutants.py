@@ -46,6 +46,11 @@ MUTANTS = [
      "key_cache[src * per_block + e] = key_cache[dst * per_block + e];"),
     ("negative slot not skipped", "if (slot < 0)\n            continue;", "if (slot < -1)\n            continue;"),
     ("last token dropped", "int32_t n = b > a ? b - a : 0;", "int32_t n = b - 1 > a ? b - 1 - a : 0;"),
+    ("prefill causal bound excludes the query's own token", "int32_t n = pos + 1 > 0 ? pos + 1 : 0;",
+     "int32_t n = pos > 0 ? pos : 0;"),
+    ("prefill chunk placed at the start of the context",
+     "int32_t pos = context_lens[s] - n_s + (t - query_start[s]);",
+     "int32_t pos = (t - query_start[s]);"),
 ]
 
 PIN_TESTS = [
@@ -63,6 +68,8 @@ PIN_TESTS = [
     pins.test_reshape_and_cache_round_trip_and_untouched_rows,
     pins.test_copy_blocks_copies_whole_blocks_only,
     pins.test_copy_on_write_branch_matches_unshared_sequence,
+    lambda: pins.test_prefill_matches_causal_sdpa(4, 4, 64, pins.wl.F16),
+    pins.test_prefill_of_whole_prompt_is_causal_self_attention,
 ]
 
 

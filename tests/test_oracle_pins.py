@@ -325,3 +325,67 @@ def test_copy_on_write_branch_matches_unshared_sequence():
         alone = oracle.decode(q[b:b + 1], kc_u, vc_u, np.array([[0, 1, 2]], np.int32),
                               lens[:1], H, 0.125, dt)
         assert np.array_equal(shared[b], alone[0])
+
+
+# ---------------------------------------------------------------- chunked prefill
+def _chunks(lens, qlens):
+    qs = np.zeros(len(lens) + 1, np.int32)
+    qs[1:] = np.cumsum(qlens)
+    return qs
+
+
+def sdpa_prefill_dense(p, qchunk, qlens):
+    """torch fp64 attention with an explicit causal mask on the dense rows."""
+    S = len(p.lens)
+    Hq, d = qchunk.shape[1], qchunk.shape[2]
+    qs = _chunks(p.lens, qlens)
+    out = np.zeros(qchunk.shape)
+    for s in range(S):
+        L, n = int(p.lens[s]), int(qlens[s])
+        if n == 0:
+            continue
+        q = torch.from_numpy(to_f64(qchunk[qs[s]:qs[s + 1]], p.dtype)).permute(1, 0, 2).unsqueeze(0)
+        k = torch.from_numpy(to_f64(p.k_dense[s, :L], p.dtype)).permute(1, 0, 2).unsqueeze(0)
+        v = torch.from_numpy(to_f64(p.v_dense[s, :L], p.dtype)).permute(1, 0, 2).unsqueeze(0)
+        allowed = np.arange(L)[None, :] <= (L - n + np.arange(n))[:, None]
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(allowed),
+                                           scale=p.scale, enable_gqa=(Hq != k.shape[1]))
+        out[qs[s]:qs[s + 1]] = o[0].permute(1, 0, 2).numpy()
+    return out
+
+
+@pytest.mark.parametrize("hq,hkv,d,dtype", [(4, 4, 64, wl.F16), (8, 2, 128, wl.BF16)])
+def test_prefill_matches_causal_sdpa(hq, hkv, d, dtype):
+    rng = wl.rng_for(30)
+    lens = np.array([40, 100, 17, 64, 5], np.int32)
+    qlens = np.array([40, 33, 1, 16, 5], np.int32)   # whole prompts, chunks, one token
+    p = make_paged(rng, 5, hq, hkv, d, lens, wl.blocks_needed(lens, 16) + 3, dtype)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), hq, d), dtype)
+    got = oracle.prefill(qchunk, p.key_cache, p.value_cache, p.tables, p.lens,
+                         _chunks(lens, qlens), hkv, p.scale, dtype)
+    np.testing.assert_allclose(got, sdpa_prefill_dense(p, qchunk, qlens), rtol=0, atol=1e-12)
+
+
+def test_prefill_of_whole_prompt_is_causal_self_attention():
+    rng = wl.rng_for(31)
+    L = 70
+    p = make_paged(rng, 1, 2, 2, 64, [L], 5, wl.F16)
+    qchunk = wl.draw_values(rng, (L, 2, 64), wl.F16)
+    got = oracle.prefill(qchunk, p.key_cache, p.value_cache, p.tables, p.lens,
+                         np.array([0, L], np.int32), 2, p.scale, wl.F16)
+    q = torch.from_numpy(to_f64(qchunk, wl.F16)).permute(1, 0, 2).unsqueeze(0)
+    k = torch.from_numpy(to_f64(p.k_dense[0, :L], wl.F16)).permute(1, 0, 2).unsqueeze(0)
+    v = torch.from_numpy(to_f64(p.v_dense[0, :L], wl.F16)).permute(1, 0, 2).unsqueeze(0)
+    ref = F.scaled_dot_product_attention(q, k, v, is_causal=True, scale=p.scale)
+    np.testing.assert_allclose(got, ref[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+    # the first query row sees only token 0: its output is V[0]
+    assert np.array_equal(got[0], to_f64(p.v_dense[0, 0], wl.F16))
+
+
+def test_prefill_with_one_token_chunks_equals_decode():
+    rng = wl.rng_for(32)
+    lens = np.array([33, 1, 200], np.int32)
+    p = make_paged(rng, 3, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
+    got = oracle.prefill(p.q, p.key_cache, p.value_cache, p.tables, p.lens,
+                         np.arange(4, dtype=np.int32), 2, p.scale, wl.BF16)
+    assert np.array_equal(got, run_oracle(p))
