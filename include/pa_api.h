@@ -150,6 +150,36 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
               int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
               void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * pa_prefill - chunked-prefill attention over the paged cache.
+ *
+ * Source: "PagedAttention in vLLM: a throughput settings guide", section
+ * "Tuning Batching, Prefill, and Cache" (chunked prefill: a step fills its
+ * token budget with chunks of prompts; each chunk attends to what is cached
+ * before it).
+ *
+ * Sequence s owns query rows query_start[s] .. query_start[s + 1] - 1 of q;
+ * they are the LAST n_s = query_start[s + 1] - query_start[s] tokens of its
+ * context of L = context_lens[s] tokens, and their K/V are already in the
+ * cache (written by pa_reshape_and_cache).  Query row i of s sits at position
+ * p = L - n_s + i; for query head h (kv head h / G):
+ *   out[row][h][:] = sum_{j <= p} softmax_j(scale * q[row][h] . K_j) V_j
+ * with K_j, V_j reached through block_tables[s][j / 16] as in pa_decode.
+ * fp32 softmax; the P.V product takes P in the input dtype (tensor cores).
+ * n_s > L or L beyond the table sets PA_DEVERR_CONTEXT_LEN (clamped).
+ *
+ *   out, q        device, [num_q_tokens][num_q_heads][head_dim], dtype
+ *   query_start   device, int32 [num_seqs + 1], non-decreasing, [num_seqs] =
+ *                 num_q_tokens
+ *   max_query_len upper bound of every n_s (sizes the grid)
+ */
+int pa_prefill(void *out, const void *q, const void *key_cache, const void *value_cache,
+               const int32_t *block_tables, const int32_t *context_lens,
+               const int32_t *query_start, int32_t max_query_len, int32_t num_kv_heads,
+               float scale, int32_t num_seqs, int32_t num_q_heads, int32_t num_q_tokens,
+               int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+               int64_t num_blocks, int32_t dtype, void *stream);
+
 /* Bytes of workspace pa_decode needs for these sizes (0 when no context can
  * exceed one partition). */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,

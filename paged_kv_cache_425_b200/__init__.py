@@ -79,6 +79,8 @@ pa_decode = _sig("pa_decode", ctypes.c_int, _P, _P, _P, _P, _P, _P, _i32, _f32, 
 pa_decode_workspace_size = _sig("pa_decode_workspace_size", _sz, _i32, _i32, _i32, _i32, _i32)
 pa_decode_static_workspace = _sig("pa_decode_static_workspace", ctypes.c_int, _P, _P, _P, _P, _P,
                                   _P, _i32, _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
+pa_prefill = _sig("pa_prefill", ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _f32, _i32,
+                  _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
 pa_copy_blocks = _sig("pa_copy_blocks", ctypes.c_int, _P, _P, _P, _i32, _i32, _i32, _i32, _i64,
                       _i32, _P)
 pa_swap_blocks = _sig("pa_swap_blocks", ctypes.c_int, _P, _P, _i64, _P, _P, _i64, _P, _i32, _i32,
@@ -204,6 +206,29 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, num_kv_he
                      _dev(context_lens, "context_lens", torch.int32, 1), hkv, float(scale), S, hq,
                      d, bs, maxb, nb, dtype_code(q), ws_ptr, ws_bytes, _stream(stream)),
            "pa_decode")
+
+
+def prefill(out, q, key_cache, value_cache, block_tables, context_lens, query_start,
+            max_query_len: int, num_kv_heads: int, scale: float, stream=None):
+    """Chunked prefill: rows query_start[s]..query_start[s+1]-1 of q are the
+    last tokens of sequence s and attend causally over its paged context."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_shape(key_cache, value_cache)
+    if hkv != num_kv_heads:
+        raise ValueError("num_kv_heads does not match the cache")
+    T, hq, dq = q.shape
+    if dq != d or tuple(out.shape) != (T, hq, d) or out.dtype != q.dtype or q.dtype != key_cache.dtype:
+        raise ValueError("q / out must be [T, Hq, d] of the cache dtype")
+    S = int(context_lens.shape[0])
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or query_start.shape != (S + 1,):
+        raise ValueError("block_tables [S, max_blocks], context_lens [S], query_start [S + 1]")
+    _check(pa_prefill(_dev(out, "out"), _dev(q, "q"), _dev(key_cache, "key_cache"),
+                      _dev(value_cache, "value_cache"),
+                      _dev(block_tables, "block_tables", torch.int32, 2),
+                      _dev(context_lens, "context_lens", torch.int32, 1),
+                      _dev(query_start, "query_start", torch.int32, 1), int(max_query_len), hkv,
+                      float(scale), S, hq, T, d, bs, int(block_tables.shape[1]), nb, dtype_code(q),
+                      _stream(stream)), "pa_prefill")
 
 
 def decode_static_workspace(out, q, key_cache, value_cache, block_tables, context_lens,

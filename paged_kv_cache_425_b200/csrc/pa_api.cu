@@ -280,6 +280,63 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
                            : dispatch_decode<__nv_bfloat16>(a, head_dim, group, tmk, tmv, st);
 }
 
+int pa_prefill(void *out, const void *q, const void *key_cache, const void *value_cache,
+               const int32_t *block_tables, const int32_t *context_lens,
+               const int32_t *query_start, int32_t max_query_len, int32_t num_kv_heads,
+               float scale, int32_t num_seqs, int32_t num_q_heads, int32_t num_q_tokens,
+               int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+               int64_t num_blocks, int32_t dtype, void *stream) {
+    int rc = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_q_tokens < 0 || max_query_len < 0 ||
+        max_blocks_per_seq <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    const int group = num_q_heads / num_kv_heads;
+    if (num_seqs == 0 || num_q_tokens == 0 || max_query_len == 0) return PA_OK;
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens ||
+        !query_start)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || !aligned(q, 4) ||
+        !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(context_lens, 4) ||
+        !aligned(query_start, 4))
+        return PA_ERR_INVALID_ARG;
+    const int64_t tiles = ((int64_t)max_query_len * group + 63) / 64;
+    if (tiles > 65535 || (int64_t)num_seqs * num_kv_heads >= (int64_t(1) << 31))
+        return PA_ERR_UNSUPPORTED;
+    constexpr int STAGES = 4;
+    const size_t smem = (size_t)STAGES * 2 * kBlock * head_dim * 2 + 1024 +
+                        (size_t)max_blocks_per_seq * 4;
+    if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
+    PrefillArgs a;
+    a.out = out;
+    a.q = q;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.query_start = query_start;
+    a.num_blocks = num_blocks;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
+        !encode_cache_map(&tmv, value_cache, num_blocks, num_kv_heads, head_dim, dtype))
+        return PA_ERR_CUDA;
+    const dim3 grid(num_seqs * num_kv_heads, (unsigned)tiles);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto launch = [&](auto kernel) -> int {
+        if (!set_smem(kernel, (int)smem)) return PA_ERR_CUDA;
+        return launch_pdl(kernel, grid, dim3(128), smem, st, tmk, tmv, a);
+    };
+    if (dtype == PA_F16)
+        return head_dim == 128 ? launch(prefill_mma_kernel<__half, 128, STAGES>)
+                               : launch(prefill_mma_kernel<__half, 64, STAGES>);
+    return head_dim == 128 ? launch(prefill_mma_kernel<__nv_bfloat16, 128, STAGES>)
+                           : launch(prefill_mma_kernel<__nv_bfloat16, 64, STAGES>);
+}
+
 int pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pairs,
                    int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                    int64_t num_blocks, int32_t dtype, void *stream) {

@@ -720,6 +720,255 @@ __global__ void copy_blocks_kernel(uint4 *__restrict__ kc, uint4 *__restrict__ v
     }
 }
 
+// ------------------------------------------------------------------ chunked prefill
+// Multi-query attention of prompt chunks over the paged cache.  Sequence s's
+// query rows are the last n_s tokens of its context (their K/V already in
+// the cache); token i sits at position L_s - n_s + i and attends to keys
+// 0 .. that position.  A CTA takes 64 query rows of one (sequence, kv head):
+// row r = token (r / G), group head (r % G); each of its 4 warps owns 16
+// rows.  K / V tiles of the sequence's blocks stream through a CTA-wide
+// STAGES-deep TMA ring (full barrier: TMA bytes; empty barrier: one arrival
+// per warp), and every warp runs the FlashAttention-style inner step on
+// mma.sync m16n8k16: S = Q K^T (K through ldmatrix), causal mask and online
+// softmax in fp32 (log2 domain), then O += P V with P packed straight from
+// the S accumulators and V through ldmatrix.trans.
+struct PrefillArgs {
+    void *out;
+    const void *q;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    const int32_t *query_start;  // [S + 1]
+    long long num_blocks;
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int max_blocks_per_seq;
+    float scale_log2;
+};
+
+constexpr float kMaskedLogit = -1.0e30f;  // finite, so 2^(masked - max) is exactly 0
+
+template <typename T, int D, int STAGES>
+__global__ void __launch_bounds__(128)
+    prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const PrefillArgs a) {
+    constexpr int NW = 4, ROWS = 64, KS = D / 16, NTD = D / 8;
+    constexpr int TILE = kBlock * D * 2, STAGE = 2 * TILE;
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t full_bar[STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[STAGES];
+    uint8_t *ring = align_smem_1024(dyn_smem);
+    int32_t *s_table = reinterpret_cast<int32_t *>(ring + STAGES * STAGE);
+
+    const int G = a.num_q_heads / a.num_kv_heads;
+    const int s = blockIdx.x / a.num_kv_heads, kvh = blockIdx.x % a.num_kv_heads;
+    const int tile = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+    pdl_launch_dependents();
+    pdl_wait_prior();
+    const int q0 = a.query_start[s];
+    int n = a.query_start[s + 1] - q0;
+    int L = a.context_lens[s];
+    const int cap = a.max_blocks_per_seq * kBlock;
+    if (L < 0 || L > cap || n < 0 || n > L) {
+        if (tile == 0 && kvh == 0 && tid == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
+        L = L < 0 ? 0 : (L > cap ? cap : L);
+        n = n < 0 ? 0 : (n > L ? L : n);
+    }
+    const int rows_total = n * G;
+    if (tile * ROWS >= rows_total) return;
+    const int last_row = min(rows_total, (tile + 1) * ROWS) - 1;
+    const int nkeys = L - n + last_row / G + 1;  // keys the tile's last row sees
+    const int nblk = (nkeys + kBlock - 1) / kBlock;
+
+    // table segment of the blocks this tile reads, checked once
+    const int32_t *trow = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+    for (int i = tid; i < nblk; i += NW * 32) {
+        int b = trow[i];
+        if (b < 0 || b >= a.num_blocks) {
+            flag_error(PA_DEVERR_BLOCK_ID);
+            b = -1;
+        }
+        s_table[i] = b;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], NW);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const uint64_t policy = l2_policy_evict_first();
+    auto issue = [&](int k) {  // thread 0
+        uint64_t *b = &full_bar[k % STAGES];
+        uint8_t *dst = ring + (k % STAGES) * STAGE;
+        const int phys = s_table[k];
+        if (phys >= 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(b, STAGE);
+            const int y = (phys * a.num_kv_heads + kvh) * kBlock;
+#pragma unroll
+            for (int x = 0; x < D; x += 64) {
+                tma_load_2d_hint(dst + (x / 64) * 2048, &tmk, b, x, y, policy);
+                tma_load_2d_hint(dst + TILE + (x / 64) * 2048, &tmv, b, x, y, policy);
+            }
+        } else {
+            mbar_arrive(b);
+        }
+    };
+    int issued = nblk < STAGES ? nblk : STAGES;
+    if (tid == 0)
+        for (int k = 0; k < issued; ++k) issue(k);
+
+    // this warp's rows: g and g + 8 of rows tile*64 + warp*16 ..
+    const int rbase = tile * ROWS + warp * 16;
+    int pos[2];
+    bool rvalid[2];
+    size_t qrow[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int R = rbase + g + 8 * e;
+        rvalid[e] = R < rows_total;
+        const int i = rvalid[e] ? R / G : 0, h = rvalid[e] ? R % G : 0;
+        pos[e] = rvalid[e] ? L - n + i : -1;
+        qrow[e] = ((size_t)(q0 + i) * a.num_q_heads + (size_t)kvh * G + h) * D;
+    }
+    const int wlast = min(rbase + 15, rows_total - 1);
+    const int warp_pmax = wlast >= rbase ? L - n + wlast / G : -1;
+    // A operand (Q rows) for all k-steps
+    uint32_t qa[KS][4];
+    const uint16_t *qb = reinterpret_cast<const uint16_t *>(a.q);
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+        qa[kk][0] = rvalid[0] ? *reinterpret_cast<const uint32_t *>(qb + qrow[0] + 16 * kk + 2 * c) : 0u;
+        qa[kk][1] = rvalid[1] ? *reinterpret_cast<const uint32_t *>(qb + qrow[1] + 16 * kk + 2 * c) : 0u;
+        qa[kk][2] = rvalid[0] ? *reinterpret_cast<const uint32_t *>(qb + qrow[0] + 16 * kk + 8 + 2 * c) : 0u;
+        qa[kk][3] = rvalid[1] ? *reinterpret_cast<const uint32_t *>(qb + qrow[1] + 16 * kk + 8 + 2 * c) : 0u;
+    }
+    float o[NTD][4];
+#pragma unroll
+    for (int j = 0; j < NTD; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m[2] = {kMaskedLogit, kMaskedLogit}, l[2] = {0.f, 0.f};
+    const int k_row = (lane & 7) + 8 * (lane >> 4), k_half = (lane >> 3) & 1;
+    const int v_row = (lane & 7) + 8 * ((lane >> 3) & 1), v_half = lane >> 4;
+
+    bool dead = false;
+    int k = 0;
+    for (; k < nblk; ++k) {
+        const int st = k % STAGES;
+        const bool ok = mbar_wait_bounded(&full_bar[st], (k / STAGES) & 1, kWaitTimeoutNs);
+        if (!__all_sync(0xffffffffu, ok)) {
+            dead = true;
+            break;
+        }
+        const int key0 = k * kBlock;
+        if (key0 <= warp_pmax && s_table[k] >= 0) {
+            const uint32_t kt = smem_addr(ring + st * STAGE), vt = kt + TILE;
+            float sf[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                uint32_t b[4];
+                ldmatrix_x4(b, kt + tile_off(k_row, 2 * kk + k_half));
+                Mma<T>::run(sf[0], qa[kk], b[0], b[1]);
+                Mma<T>::run(sf[1], qa[kk], b[2], b[3]);
+            }
+            // sf[nt]: (row g, keys 8nt+2c, +1), (row g+8, same keys)
+            float pv[2][4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {  // row g (e = 0) / g + 8 (e = 1)
+                float x[4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int key = key0 + 8 * nt + 2 * c + u;
+                        x[2 * nt + u] = key <= pos[e] ? sf[nt][2 * e + u] * a.scale_log2 : kMaskedLogit;
+                    }
+                float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+                bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+                bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+                const float m_new = fmaxf(m[e], bm);
+                const float alpha = fast_exp2(m[e] - m_new);
+                float sum = 0.f;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    x[t] = fast_exp2(x[t] - m_new);
+                    sum += x[t];
+                }
+                l[e] = l[e] * alpha + sum;
+                m[e] = m_new;
+#pragma unroll
+                for (int j = 0; j < NTD; ++j) {
+                    o[j][2 * e] *= alpha;
+                    o[j][2 * e + 1] *= alpha;
+                }
+                pv[0][2 * e] = x[0]; pv[0][2 * e + 1] = x[1];
+                pv[1][2 * e] = x[2]; pv[1][2 * e + 1] = x[3];
+            }
+            uint32_t pa[4];
+            pa[0] = Mma<T>::pack(pv[0][0], pv[0][1]);  // row g,     keys 2c..
+            pa[1] = Mma<T>::pack(pv[0][2], pv[0][3]);  // row g + 8, keys 2c..
+            pa[2] = Mma<T>::pack(pv[1][0], pv[1][1]);  // row g,     keys 8 + 2c..
+            pa[3] = Mma<T>::pack(pv[1][2], pv[1][3]);  // row g + 8, keys 8 + 2c..
+            // keys past the context (last block) may hold anything: zero
+            // their V entries in the fragments
+            const int nvalid = min(kBlock, L - key0);
+#pragma unroll
+            for (int j = 0; j < NTD; j += 2) {
+                uint32_t b[4];
+                ldmatrix_x4_trans(b, vt + tile_off(v_row, j + v_half));
+                if (nvalid < kBlock) {
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int kb = 8 * (r & 1) + 2 * c;
+                        if (kb >= nvalid) b[r] &= 0xffff0000u;
+                        if (kb + 1 >= nvalid) b[r] &= 0x0000ffffu;
+                    }
+                }
+                Mma<T>::run(o[j], pa, b[0], b[1]);
+                Mma<T>::run(o[j + 1], pa, b[2], b[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);
+        if (warp == 0 && issued < nblk) {
+            // refill this stage once every warp has released it
+            const bool freed = mbar_wait_bounded(&empty_bar[st], (k / STAGES) & 1, kWaitTimeoutNs);
+            if (!__all_sync(0xffffffffu, freed)) {
+                dead = true;
+                ++k;
+                break;
+            }
+            if (lane == 0) issue(issued);
+            ++issued;
+        }
+    }
+    if (dead) {
+        // wait (bounded) for loads still in flight before the CTA exits
+        for (int j = k; j < issued; ++j)
+            if (!mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1, kWaitTimeoutNs)) break;
+        return;
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        l[e] += __shfl_xor_sync(0xffffffffu, l[e], 1);
+        l[e] += __shfl_xor_sync(0xffffffffu, l[e], 2);
+    }
+    uint16_t *ob = reinterpret_cast<uint16_t *>(a.out);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        if (!rvalid[e]) continue;
+        const float inv = l[e] > 0.f ? 1.f / l[e] : 0.f;
+#pragma unroll
+        for (int j = 0; j < NTD; ++j) {
+            const uint32_t packed =
+                (uint32_t)narrow1(o[j][2 * e] * inv, T()) | ((uint32_t)narrow1(o[j][2 * e + 1] * inv, T()) << 16);
+            *reinterpret_cast<uint32_t *>(ob + qrow[e] + 8 * j + 2 * c) = packed;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ block swap
 // Whole blocks between two pools, either of which may be mapped page-locked
 // host memory reached through its device alias: grid.x strides over pairs,

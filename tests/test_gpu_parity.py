@@ -378,3 +378,73 @@ def test_swap_out_and_back_in_is_bit_exact_and_decode_follows(pinned):
     with pytest.raises(pk.PagedError) as e:
         pk.swap_blocks(dkc, dvc, host_k, host_v, np.array([[0, 40]], np.int32))
     assert e.value.status == pk.PA_ERR_OUT_OF_RANGE
+
+
+# ---------------------------------------------------------------- chunked prefill
+def run_prefill(p, qchunk, qlens, max_query_len=None):
+    qs = np.zeros(len(qlens) + 1, np.int32)
+    qs[1:] = np.cumsum(qlens)
+    q = gh.to_dev(qchunk, p.dtype)
+    out = torch.full_like(q, float("nan"))
+    pk.prefill(out, q, gh.to_dev(p.key_cache, p.dtype), gh.to_dev(p.value_cache, p.dtype),
+               gh.ints(p.tables), gh.ints(p.lens), gh.ints(qs),
+               int(max(qlens)) if max_query_len is None else max_query_len, p.num_kv_heads,
+               p.scale)
+    torch.cuda.synchronize()
+    ref = oracle.prefill(qchunk, p.key_cache, p.value_cache, p.tables, p.lens, qs,
+                         p.num_kv_heads, p.scale, p.dtype)
+    return out, ref
+
+
+@pytest.mark.parametrize("hq,hkv,d,dtype", [(4, 4, 64, wl.F16), (8, 2, 128, wl.BF16),
+                                            (32, 8, 128, wl.BF16), (8, 1, 64, wl.F16),
+                                            (16, 16, 128, wl.F16)])
+def test_prefill_matches_oracle(hq, hkv, d, dtype):
+    rng = wl.rng_for(40 + hq + d)
+    lens = np.array([40, 700, 17, 64, 5, 1, 513], np.int32)
+    qlens = np.array([40, 300, 1, 16, 5, 1, 77], np.int32)  # whole prompts, chunks, single tokens
+    p = make_paged(rng, len(lens), hq, hkv, d, lens, wl.blocks_needed(lens, 16) + 3, dtype)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), hq, d), dtype)
+    out, ref = run_prefill(p, qchunk, qlens)
+    assert pk.get_error() == (0, 0)
+    assert gh.max_err(out, ref) <= gh.TOL[dtype]
+
+
+def test_prefill_one_token_chunks_agree_with_decode():
+    rng = wl.rng_for(41)
+    lens = np.array([33, 1, 1200, 512], np.int32)
+    p = make_paged(rng, 4, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
+    out, ref = run_prefill(p, p.q, np.ones(4, np.int32))
+    dec = gpu_out(p)
+    assert gh.max_err(out, ref) <= gh.TOL[wl.BF16]
+    assert float((out.float() - dec.float()).abs().max()) <= gh.TOL[wl.BF16]
+
+
+def test_prefill_long_contexts_and_slack_grid():
+    """Chunks of 512 over contexts up to 4k, with a grid sized for a larger
+    max_query_len than any sequence uses."""
+    rng = wl.rng_for(42)
+    lens = np.array([4096, 1024, 2600], np.int32)
+    qlens = np.array([512, 512, 100], np.int32)
+    p = make_paged(rng, 3, 32, 8, 128, lens, wl.blocks_needed(lens, 16) + 1, wl.BF16)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), 32, 128), wl.BF16)
+    out, ref = run_prefill(p, qchunk, qlens, max_query_len=900)
+    assert gh.max_err(out, ref) <= gh.TOL[wl.BF16]
+
+
+def test_prefill_chunk_longer_than_context_is_reported():
+    rng = wl.rng_for(43)
+    lens = np.array([20, 30], np.int32)
+    p = make_paged(rng, 2, 4, 4, 64, lens, 4, wl.F16)
+    qlens = np.array([25, 30], np.int32)  # 25 > 20: clamped, flagged
+    qchunk = wl.draw_values(rng, (55, 4, 64), wl.F16)
+    qs = np.array([0, 25, 55], np.int32)
+    q = gh.to_dev(qchunk, wl.F16)
+    out = torch.zeros_like(q)
+    pk.prefill(out, q, gh.to_dev(p.key_cache, wl.F16), gh.to_dev(p.value_cache, wl.F16),
+               gh.ints(p.tables), gh.ints(p.lens), gh.ints(qs), 30, 4, p.scale)
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_CONTEXT_LEN
+    ref = oracle.prefill(qchunk[25:], p.key_cache, p.value_cache, p.tables[1:], p.lens[1:],
+                         np.array([0, 30], np.int32), 4, p.scale, wl.F16)
+    assert gh.max_err(out[25:], ref) <= gh.TOL[wl.F16]
