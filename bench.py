@@ -49,7 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b",
-                    choices=["llama7b", "llama13b", "gqa_long", "cow", "tiny", "swap"])
+                    choices=["llama7b", "llama13b", "gqa_long", "cow", "tiny", "swap", "prefill"])
     ap.add_argument("--layers", type=int, default=0,
                     help="layer caches to allocate (0: the workload's layer count; fewer "
                          "caches are cycled so every step still runs every layer)")
@@ -533,6 +533,127 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def prefill_flops(lens, chunk, num_q_heads, head_dim):
+    """Multiply-adds x 2 of chunked prefill: query token i of a sequence with
+    context L attends to L - chunk + i + 1 keys, for q.K and for P.V."""
+    total = 0
+    for L in np.asarray(lens, dtype=np.int64):
+        n = min(chunk, int(L))
+        keys = (L - n + 1) * n + n * (n - 1) // 2
+        total += 4 * int(keys) * head_dim * num_q_heads
+    return total
+
+
+def run_prefill(args, world, rank, local):
+    """Chunked-prefill step: for each of 32 layers, pa_reshape_and_cache of
+    the step's 16 x 512 chunk tokens, then pa_prefill over the paged cache."""
+    import torch
+    import paged_kv_cache_425_b200 as pk
+    from paged_kv_cache_425_b200 import batch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    w = wl.WORKLOADS["prefill"]
+    if args.num_seqs:
+        w = wl.scaled(w, num_seqs=args.num_seqs)
+    rng = wl.rng_for(args.seed + rank)
+    lens = wl.draw_context_lens(w, rng)
+    nb = wl.pool_size(w, lens)
+    a = batch.scattered_allocator(nb, wl.draw_block_order(nb, rng))
+    chunk = w.chunk
+    slots = []
+    for s_, L in enumerate(lens):
+        a.add_seq(s_, int(L) - chunk)            # context cached before this step
+        sl, _ = a.append_slots(np.full(chunk, s_, np.int64))
+        slots.append(sl)                         # the chunk's own slots
+    maxb = batch.max_blocks_for(w)
+    tables, ctx = a.build_tables(np.arange(len(lens)), maxb)
+    T = chunk * len(lens)
+    H, Hq, d = w.num_kv_heads, w.num_q_heads, w.head_dim
+    layers = w.layers
+    ncache = min(args.layers if args.layers > 0 else layers, layers)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2000 + args.seed + rank)
+    tdt = torch.bfloat16 if w.dtype == wl.BF16 else torch.float16
+    kc = [torch.randn((nb, H, 16, d), generator=gen, device=device, dtype=tdt) for _ in range(ncache)]
+    vc = [torch.randn((nb, H, 16, d), generator=gen, device=device, dtype=tdt) for _ in range(ncache)]
+    q = torch.randn((layers, T, Hq, d), generator=gen, device=device, dtype=tdt)
+    kn = torch.randn((layers, T, H, d), generator=gen, device=device, dtype=tdt)
+    vn = torch.randn((layers, T, H, d), generator=gen, device=device, dtype=tdt)
+    out = torch.empty_like(q)
+    d_tables = torch.from_numpy(tables).to(device)
+    d_lens = torch.from_numpy(ctx).to(device)
+    d_qs = torch.from_numpy(np.arange(0, T + 1, chunk, dtype=np.int32)).to(device)
+    d_slots = torch.from_numpy(np.concatenate(slots)).to(device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        for l in range(layers):
+            c = l % ncache
+            pk.reshape_and_cache(kn[l], vn[l], kc[c], vc[c], d_slots, stream=stream)
+            if ev is not None:
+                ev[0][l].record(stream)
+            pk.prefill(out[l], q[l], kc[c], vc[c], d_tables, d_lens, d_qs, chunk, H, w.scale,
+                       stream=stream)
+            if ev is not None:
+                ev[1][l].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    rc, bits = pk.get_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error word {bits:#x}")
+    sampler = ClockSampler(device)
+    barrier(device)
+    torch.cuda.synchronize()
+    sampler.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = []
+    t0.record(stream)
+    for _ in range(args.steps):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(layers)] for _ in range(2)]
+        step(ev)
+        evs.append(ev)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), device)
+    call_ms = max_over_ranks(float(np.mean([x.elapsed_time(y) for ev in evs
+                                            for x, y in zip(ev[0], ev[1])])), device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    flops = prefill_flops(ctx, chunk, Hq, d)
+    tflops = flops / (call_ms * 1e-3) / 1e12
+    try:
+        with open(PEAKS_FILE) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+        src = "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    line = {
+        "metric": "chunked-prefill attention query tokens/s and achieved TFLOP/s",
+        "value": round(world * T * args.steps / (total_ms * 1e-3), 1), "unit": "query tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**describe(w, ctx, ncache), "chunk": chunk, "query_tokens_per_step_layer": T},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                     "kernel": "prefill_mma_kernel (mma.sync m16n8k16)", "flops_per_call": flops,
+                     "avg_call_us": round(call_ms * 1e3, 2), "peak_source": src},
+        "gpu_launches": args.steps * layers * 2,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_swap(args):
     """Swap bandwidth: scattered blocks of the Llama-7B layer shape (32 kv
     heads x 16 x 128, fp16; 128 KiB per K or V block) between the device
@@ -584,9 +705,17 @@ def main(argv=None):
         if rank == 0:
             run_swap(args)
         return 0
+    if args.workload == "prefill" and args.impl == "ours":
+        run_prefill(args, world, rank, local)
+        return 0
     if world > 1 and args.gpus != world:
         args.gpus = world
     if args.impl == "reference":
+        if args.workload in ("swap", "prefill"):
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "the CPU reference arm times decode workloads only"}))
+            return 0
         run_reference(args, world, rank)
         return 0
     run_ours(args, world, rank, local)

@@ -319,6 +319,7 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
     a.num_q_heads = num_q_heads;
     a.num_kv_heads = num_kv_heads;
     a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_q_tokens = num_q_tokens;
     a.scale_log2 = scale * 1.4426950408889634f;
     CUtensorMap tmk, tmv;
     if (!encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||

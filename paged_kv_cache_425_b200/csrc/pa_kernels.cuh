@@ -743,6 +743,7 @@ struct PrefillArgs {
     int num_q_heads;
     int num_kv_heads;
     int max_blocks_per_seq;
+    int num_q_tokens;
     float scale_log2;
 };
 
@@ -770,6 +771,10 @@ __global__ void __launch_bounds__(128)
     int n = a.query_start[s + 1] - q0;
     int L = a.context_lens[s];
     const int cap = a.max_blocks_per_seq * kBlock;
+    if (q0 < 0 || q0 > a.num_q_tokens || n > a.num_q_tokens - q0) {  // rows outside q / out
+        if (tile == 0 && kvh == 0 && tid == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
+        return;
+    }
     if (L < 0 || L > cap || n < 0 || n > L) {
         if (tile == 0 && kvh == 0 && tid == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
         L = L < 0 ? 0 : (L > cap ? cap : L);

@@ -52,6 +52,8 @@ class Workload:
     branches: int = 0
     prompt_len: int = 0
     own_max: int = 0
+    # chunked prefill: every sequence's last `chunk` tokens are the query chunk
+    chunk: int = 0
 
     @property
     def scale(self) -> float:
@@ -71,6 +73,9 @@ WORKLOADS = {
     # parallel sampling: 32 prompts x 4 branches of a 1000-token prompt
     "cow": Workload("cow", 128, 32, 32, 128, 16, BF16, 32, ("fixed", 1000), prompts=32, branches=4,
                     prompt_len=1000, own_max=256),
+    # chunked prefill: 16 seqs x 512-token chunks (an 8192-token step budget)
+    # over contexts U{512..4096}, Llama-3.1-8B shape (32 q / 8 kv heads, bf16)
+    "prefill": Workload("prefill", 16, 32, 8, 128, 16, BF16, 32, ("uniform", 512, 4096), chunk=512),
 }
 
 
