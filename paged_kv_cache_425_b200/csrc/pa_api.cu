@@ -132,8 +132,9 @@ int launch_decode(const DecodeArgs &a, int group, const CUtensorMap &tmk, const 
         rc = launch_pdl(k, grid, block, SMEM, st, tmk, tmv, a);
     }
     if (rc != PA_OK || a.num_parts <= 1) return rc;
-    return launch_pdl(merge_kernel<T, D>, dim3(a.num_seqs * a.num_q_heads), dim3(kMergeThreads),
-                      a.num_parts * sizeof(float), st, a);
+    const int64_t rows = (int64_t)a.num_seqs * a.num_q_heads;
+    return launch_pdl(merge_kernel<T, D>, dim3((unsigned)((rows + kMergeRows - 1) / kMergeRows)),
+                      dim3(kMergeRows * 32), 0, st, a);
 }
 
 template <typename T>

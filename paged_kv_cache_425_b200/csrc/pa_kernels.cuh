@@ -598,69 +598,64 @@ __global__ void __launch_bounds__(NW * 32)
 }
 
 // ------------------------------------------------------------------ partition merge
-// One CTA of kMergeThreads per (sequence, q head) whose context spans more
-// than one partition: out = sum_p w_p o_p / sum_p w_p, w_p = l_p 2^(m_p - M),
-// M = max over partitions that saw a token.  Weights go to shared memory
-// first; the partial outputs then stream in as independent coalesced loads.
-constexpr int kMergeThreads = 128;
+// One warp per (sequence, q head) whose context spans more than one
+// partition, kMergeRows rows per CTA: out = sum_p w_p o_p / sum_p w_p with
+// w_p = l_p 2^(m_p - M), M = max over partitions that saw a token.  Lane i
+// owns partitions i, i + 32, ... for the weights and elements 4i .. 4i + 3 of
+// the row (D / 4 lanes) for the sum; weights travel by shuffle, the partial
+// rows stream in as independent 16-byte loads.  No block barrier.
+constexpr int kMergeRows = 4;
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
-    extern __shared__ float s_w[];  // [num_parts]
-    __shared__ float s_red[kMergeThreads / 32];
-    __shared__ float s_bcast;
+__global__ void __launch_bounds__(kMergeRows * 32) merge_kernel(const DecodeArgs a) {
     pdl_launch_dependents();
     pdl_wait_prior();
-    const int row = blockIdx.x;
-    const int s = row / a.num_q_heads;
+    const int lane = threadIdx.x & 31;
+    const size_t row = (size_t)blockIdx.x * kMergeRows + (threadIdx.x >> 5);
+    if (row >= (size_t)a.num_seqs * a.num_q_heads) return;
+    const int s = (int)(row / a.num_q_heads);
     const int L = clamp_context(a, s, false);
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
     if (nparts <= 1) return;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const float2 *ml = a.ws_ml + (size_t)row * a.num_parts;
-
+    const float2 *ml = a.ws_ml + row * a.num_parts;
     float M = -INFINITY;
-    for (int p = threadIdx.x; p < nparts; p += kMergeThreads) {
+    for (int p = lane; p < nparts; p += 32) {
         const float2 v = ml[p];
         if (v.y > 0.f) M = fmaxf(M, v.x);
     }
+#pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) s_red[warp] = M;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float v = s_red[0];
-        for (int w = 1; w < kMergeThreads / 32; ++w) v = fmaxf(v, s_red[w]);
-        s_bcast = v;
-    }
-    __syncthreads();
-    M = s_bcast;
+    constexpr int D4 = D / 4;  // float4 pieces of a row
+    const float4 *op = reinterpret_cast<const float4 *>(a.ws_o + row * a.num_parts * D);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float den = 0.f;
-    for (int p = threadIdx.x; p < nparts; p += kMergeThreads) {
-        const float2 v = ml[p];
-        const float w = v.y > 0.f ? v.y * fast_exp2(v.x - M) : 0.f;
-        s_w[p] = w;
+    for (int p0 = 0; p0 < nparts; p0 += 32) {
+        const int p = p0 + lane;
+        float w = 0.f;
+        if (p < nparts) {
+            const float2 v = ml[p];
+            w = v.y > 0.f ? v.y * fast_exp2(v.x - M) : 0.f;
+        }
         den += w;
+        const int cnt = min(32, nparts - p0);
+#pragma unroll 4
+        for (int j = 0; j < cnt; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            if (lane < D4) {
+                const float4 x = op[(size_t)(p0 + j) * D4 + lane];
+                acc.x += wj * x.x; acc.y += wj * x.y; acc.z += wj * x.z; acc.w += wj * x.w;
+            }
+        }
     }
+#pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    __syncthreads();  // every thread has read s_bcast; s_red is free again
-    if (lane == 0) s_red[warp] = den;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float v = 0.f;
-        for (int w = 0; w < kMergeThreads / 32; ++w) v += s_red[w];
-        s_bcast = v;
-    }
-    __syncthreads();
-    den = s_bcast;
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    const float *o_parts = a.ws_o + (size_t)row * a.num_parts * D;
-    uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + (size_t)row * D;
-    for (int d = threadIdx.x; d < D; d += kMergeThreads) {
-        float o = 0.f;
-#pragma unroll 8
-        for (int p = 0; p < nparts; ++p) o += s_w[p] * o_parts[(size_t)p * D + d];
-        out[d] = narrow1(o * inv, T());
+    if (lane < D4) {
+        uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + row * D + 4 * lane;
+        const uint32_t lo = (uint32_t)narrow1(acc.x * inv, T()) | ((uint32_t)narrow1(acc.y * inv, T()) << 16);
+        const uint32_t hi = (uint32_t)narrow1(acc.z * inv, T()) | ((uint32_t)narrow1(acc.w * inv, T()) << 16);
+        *reinterpret_cast<uint2 *>(out) = make_uint2(lo, hi);
     }
 }
 
@@ -879,7 +874,7 @@ __global__ void __launch_bounds__(128)
                 Mma<T>::run(sf[1], qa[kk], b[2], b[3]);
             }
             // sf[nt]: (row g, keys 8nt+2c, +1), (row g+8, same keys)
-            float pv[2][4];
+            float pv[2][4], alpha_row[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {  // row g (e = 0) / g + 8 (e = 1)
                 float x[4];
@@ -903,13 +898,20 @@ __global__ void __launch_bounds__(128)
                 }
                 l[e] = l[e] * alpha + sum;
                 m[e] = m_new;
-#pragma unroll
-                for (int j = 0; j < NTD; ++j) {
-                    o[j][2 * e] *= alpha;
-                    o[j][2 * e + 1] *= alpha;
-                }
+                alpha_row[e] = alpha;
                 pv[0][2 * e] = x[0]; pv[0][2 * e + 1] = x[1];
                 pv[1][2 * e] = x[2]; pv[1][2 * e + 1] = x[3];
+            }
+            // rescale the accumulators only when some row of the warp raised
+            // its running max (alpha < 1); once the max settles this is skipped
+            if (__any_sync(0xffffffffu, alpha_row[0] != 1.f || alpha_row[1] != 1.f)) {
+#pragma unroll
+                for (int j = 0; j < NTD; ++j) {
+                    o[j][0] *= alpha_row[0];
+                    o[j][1] *= alpha_row[0];
+                    o[j][2] *= alpha_row[1];
+                    o[j][3] *= alpha_row[1];
+                }
             }
             uint32_t pa[4];
             pa[0] = Mma<T>::pack(pv[0][0], pv[0][1]);  // row g,     keys 2c..
