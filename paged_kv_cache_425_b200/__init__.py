@@ -301,6 +301,7 @@ class BlockAllocator:
     """Host block allocator (free list, refcounts, copy-on-write) of libpa.so."""
 
     def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE):
+        self._destroy = pa_alloc_destroy  # kept: module globals may be gone at exit
         self._h = pa_alloc_create(num_blocks, block_size)
         if not self._h:
             raise ValueError("bad pool size")
@@ -310,7 +311,7 @@ class BlockAllocator:
     def __del__(self):
         h = getattr(self, "_h", None)
         if h:
-            pa_alloc_destroy(h)
+            self._destroy(h)
             self._h = None
 
     def add_seq(self, seq_id: int, num_tokens: int):

@@ -853,54 +853,79 @@ __global__ void __launch_bounds__(128)
     const int k_row = (lane & 7) + 8 * (lane >> 4), k_half = (lane >> 3) & 1;
     const int v_row = (lane & 7) + 8 * ((lane >> 3) & 1), v_half = lane >> 4;
 
+    // Two 16-key blocks per step: the softmax and the rescale check are paid
+    // once per 32 keys.
     bool dead = false;
     int k = 0;
-    for (; k < nblk; ++k) {
-        const int st = k % STAGES;
-        const bool ok = mbar_wait_bounded(&full_bar[st], (k / STAGES) & 1, kWaitTimeoutNs);
+    for (; k < nblk; k += 2) {
+        const bool two = k + 1 < nblk;
+        bool ok = mbar_wait_bounded(&full_bar[k % STAGES], (k / STAGES) & 1, kWaitTimeoutNs);
+        if (two)
+            ok = mbar_wait_bounded(&full_bar[(k + 1) % STAGES], ((k + 1) / STAGES) & 1,
+                                   kWaitTimeoutNs) && ok;
         if (!__all_sync(0xffffffffu, ok)) {
             dead = true;
             break;
         }
         const int key0 = k * kBlock;
-        if (key0 <= warp_pmax && s_table[k] >= 0) {
-            const uint32_t kt = smem_addr(ring + st * STAGE), vt = kt + TILE;
-            float sf[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        bool use[2];
+        use[0] = s_table[k] >= 0 && key0 <= warp_pmax;
+        use[1] = two && s_table[k + 1] >= 0 && key0 + kBlock <= warp_pmax;
+        if (use[0] || use[1]) {
+            uint32_t kt[2], vt[2];
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                kt[bb] = smem_addr(ring + ((k + bb) % STAGES) * STAGE);
+                vt[bb] = kt[bb] + TILE;
+            }
+            // sf[2 bb + nt]: block k + bb, keys 8 nt + 2c (+1); rows g / g + 8
+            float sf[4][4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) sf[t][0] = sf[t][1] = sf[t][2] = sf[t][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
-                uint32_t b[4];
-                ldmatrix_x4(b, kt + tile_off(k_row, 2 * kk + k_half));
-                Mma<T>::run(sf[0], qa[kk], b[0], b[1]);
-                Mma<T>::run(sf[1], qa[kk], b[2], b[3]);
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    if (!use[bb]) continue;
+                    uint32_t b[4];
+                    ldmatrix_x4(b, kt[bb] + tile_off(k_row, 2 * kk + k_half));
+                    Mma<T>::run(sf[2 * bb], qa[kk], b[0], b[1]);
+                    Mma<T>::run(sf[2 * bb + 1], qa[kk], b[2], b[3]);
+                }
             }
-            // sf[nt]: (row g, keys 8nt+2c, +1), (row g+8, same keys)
-            float pv[2][4], alpha_row[2];
+            float pv[4][4], alpha_row[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {  // row g (e = 0) / g + 8 (e = 1)
-                float x[4];
+                float x[8];
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int t = 0; t < 4; ++t)
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int key = key0 + 8 * nt + 2 * c + u;
-                        x[2 * nt + u] = key <= pos[e] ? sf[nt][2 * e + u] * a.scale_log2 : kMaskedLogit;
+                        const int key = key0 + 8 * t + 2 * c + u;
+                        x[2 * t + u] = (use[t >> 1] && key <= pos[e])
+                                           ? sf[t][2 * e + u] * a.scale_log2 : kMaskedLogit;
                     }
-                float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+                float bm = x[0];
+#pragma unroll
+                for (int t = 1; t < 8; ++t) bm = fmaxf(bm, x[t]);
                 bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
                 bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
                 const float m_new = fmaxf(m[e], bm);
                 const float alpha = fast_exp2(m[e] - m_new);
                 float sum = 0.f;
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
+                for (int t = 0; t < 8; ++t) {
                     x[t] = fast_exp2(x[t] - m_new);
                     sum += x[t];
                 }
                 l[e] = l[e] * alpha + sum;
                 m[e] = m_new;
                 alpha_row[e] = alpha;
-                pv[0][2 * e] = x[0]; pv[0][2 * e + 1] = x[1];
-                pv[1][2 * e] = x[2]; pv[1][2 * e + 1] = x[3];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    pv[t][2 * e] = x[2 * t];
+                    pv[t][2 * e + 1] = x[2 * t + 1];
+                }
             }
             // rescale the accumulators only when some row of the warp raised
             // its running max (alpha < 1); once the max settles this is skipped
@@ -913,42 +938,55 @@ __global__ void __launch_bounds__(128)
                     o[j][3] *= alpha_row[1];
                 }
             }
-            uint32_t pa[4];
-            pa[0] = Mma<T>::pack(pv[0][0], pv[0][1]);  // row g,     keys 2c..
-            pa[1] = Mma<T>::pack(pv[0][2], pv[0][3]);  // row g + 8, keys 2c..
-            pa[2] = Mma<T>::pack(pv[1][0], pv[1][1]);  // row g,     keys 8 + 2c..
-            pa[3] = Mma<T>::pack(pv[1][2], pv[1][3]);  // row g + 8, keys 8 + 2c..
-            // keys past the context (last block) may hold anything: zero
-            // their V entries in the fragments
-            const int nvalid = min(kBlock, L - key0);
 #pragma unroll
-            for (int j = 0; j < NTD; j += 2) {
-                uint32_t b[4];
-                ldmatrix_x4_trans(b, vt + tile_off(v_row, j + v_half));
-                if (nvalid < kBlock) {
+            for (int bb = 0; bb < 2; ++bb) {
+                if (!use[bb]) continue;
+                uint32_t pa[4];
+                pa[0] = Mma<T>::pack(pv[2 * bb][0], pv[2 * bb][1]);          // row g,     keys 2c..
+                pa[1] = Mma<T>::pack(pv[2 * bb][2], pv[2 * bb][3]);          // row g + 8, keys 2c..
+                pa[2] = Mma<T>::pack(pv[2 * bb + 1][0], pv[2 * bb + 1][1]);  // row g,     keys 8 + 2c..
+                pa[3] = Mma<T>::pack(pv[2 * bb + 1][2], pv[2 * bb + 1][3]);  // row g + 8, keys 8 + 2c..
+                // keys past the context (last block) may hold anything: zero
+                // their V entries in the fragments
+                const int nvalid = min(kBlock, L - (key0 + kBlock * bb));
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int kb = 8 * (r & 1) + 2 * c;
-                        if (kb >= nvalid) b[r] &= 0xffff0000u;
-                        if (kb + 1 >= nvalid) b[r] &= 0x0000ffffu;
+                for (int j = 0; j < NTD; j += 2) {
+                    uint32_t b[4];
+                    ldmatrix_x4_trans(b, vt[bb] + tile_off(v_row, j + v_half));
+                    if (nvalid < kBlock) {
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int kb = 8 * (r & 1) + 2 * c;
+                            if (kb >= nvalid) b[r] &= 0xffff0000u;
+                            if (kb + 1 >= nvalid) b[r] &= 0x0000ffffu;
+                        }
                     }
+                    Mma<T>::run(o[j], pa, b[0], b[1]);
+                    Mma<T>::run(o[j + 1], pa, b[2], b[3]);
                 }
-                Mma<T>::run(o[j], pa, b[0], b[1]);
-                Mma<T>::run(o[j + 1], pa, b[2], b[3]);
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[st]);
-        if (warp == 0 && issued < nblk) {
-            // refill this stage once every warp has released it
-            const bool freed = mbar_wait_bounded(&empty_bar[st], (k / STAGES) & 1, kWaitTimeoutNs);
-            if (!__all_sync(0xffffffffu, freed)) {
-                dead = true;
-                ++k;
+        if (lane == 0) {
+            mbar_arrive(&empty_bar[k % STAGES]);
+            if (two) mbar_arrive(&empty_bar[(k + 1) % STAGES]);
+        }
+        if (warp == 0) {
+            // refill the consumed stages once every warp has released them
+            for (int kb = k; kb < k + (two ? 2 : 1) && issued < nblk; ++kb) {
+                const bool freed =
+                    mbar_wait_bounded(&empty_bar[kb % STAGES], (kb / STAGES) & 1, kWaitTimeoutNs);
+                if (!__all_sync(0xffffffffu, freed)) {
+                    dead = true;
+                    break;
+                }
+                if (lane == 0) issue(issued);
+                ++issued;
+            }
+            if (dead) {
+                k += two ? 2 : 1;
                 break;
             }
-            if (lane == 0) issue(issued);
-            ++issued;
         }
     }
     if (dead) {
