@@ -438,7 +438,17 @@ def run_e2e(st, args, device, world, chunks: int = 4):
     ev_meta_free = torch.cuda.Event()
     first = [True]
 
-    def one():
+    def one_serial():
+        with torch.cuda.stream(comp):
+            for dev, host in meta:
+                dev.copy_(host, non_blocking=True)
+            st.q.copy_(hq, non_blocking=True)
+            st.k_new.copy_(hk, non_blocking=True)
+            st.v_new.copy_(hv, non_blocking=True)
+            st.step()
+            hout.copy_(st.out, non_blocking=True)
+
+    def one_overlapped():
         with torch.cuda.stream(copy):
             if not first[0]:
                 copy.wait_event(ev_meta_free)
@@ -468,6 +478,9 @@ def run_e2e(st, args, device, world, chunks: int = 4):
         comp.wait_event(ev_read[-1])                  # the step ends when its outputs are back
         first[0] = False
 
+    # with one layer group there is nothing to overlap: one stream, no syncs
+    one = one_overlapped if len(groups) > 1 else one_serial
+
     for _ in range(max(1, args.warmup)):
         one()
     barrier(device)
@@ -486,7 +499,8 @@ def run_e2e(st, args, device, world, chunks: int = 4):
     return {"value": round(world * st.S * args.steps / (ms * 1e-3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms / args.steps, 4),
-            "overlap": f"copy stream, {len(groups)} layer groups"}
+            "overlap": (f"copy stream, {len(groups)} layer groups" if len(groups) > 1
+                        else "none (one layer): copies and kernels on one stream")}
 
 
 # ---------------------------------------------------------------- CPU oracle
