@@ -121,3 +121,43 @@ def test_cow_divergence_and_following_steps_full_size():
         assert gh.max_err(out[torch.from_numpy(sel).long().cuda()], ref) <= gh.TOL[w.dtype]
     assert np.array_equal(gh.to_host_bits(dkc), kc)
     assert np.array_equal(gh.to_host_bits(dvc), vc)
+
+
+def test_prefill_workload_full_size_sampled_sequences():
+    """16 sequences x 512-token chunks over contexts U{512..4096} (32 q / 8 kv
+    heads, bf16), tables from the allocator as in bench.py; the chunk's own
+    K/V written by pa_reshape_and_cache, then pa_prefill; the oracle checks
+    three whole sequences (every query row of them)."""
+    w = wl.WORKLOADS["prefill"]
+    rng = wl.rng_for(0)
+    lens = wl.draw_context_lens(w, rng)
+    nb = wl.pool_size(w, lens)
+    a = batch.scattered_allocator(nb, wl.draw_block_order(nb, rng))
+    slots = []
+    for s, L in enumerate(lens):
+        a.add_seq(s, int(L) - w.chunk)
+        sl, _ = a.append_slots(np.full(w.chunk, s, np.int64))
+        slots.append(sl)
+    tables, ctx = a.build_tables(np.arange(len(lens)), batch.max_blocks_for(w))
+    slots = np.concatenate(slots)
+    T = w.chunk * len(lens)
+    H, Hq, d, dt = w.num_kv_heads, w.num_q_heads, w.head_dim, w.dtype
+    kc, vc = host_pool(rng, nb, w)
+    q = wl.draw_values(rng, (T, Hq, d), dt)
+    k_new = wl.draw_values(rng, (T, H, d), dt)
+    v_new = wl.draw_values(rng, (T, H, d), dt)
+    dkc, dvc = gh.to_dev(kc, dt), gh.to_dev(vc, dt)
+    pk.reshape_and_cache(gh.to_dev(k_new, dt), gh.to_dev(v_new, dt), dkc, dvc,
+                         gh.ints(slots, torch.int64))
+    oracle.reshape_and_cache(k_new, v_new, kc, vc, slots)
+    qs = np.arange(0, T + 1, w.chunk, dtype=np.int32)
+    out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device="cuda")
+    pk.prefill(out, gh.to_dev(q, dt), dkc, dvc, gh.ints(tables), gh.ints(ctx), gh.ints(qs),
+               w.chunk, H, w.scale)
+    torch.cuda.synchronize()
+    assert pk.get_error() == (0, 0)
+    for s in (int(np.argmax(ctx)), int(np.argmin(ctx)), 5):
+        sl = slice(s * w.chunk, (s + 1) * w.chunk)
+        ref = oracle.prefill(q[sl], kc, vc, tables[s:s + 1], ctx[s:s + 1],
+                             np.array([0, w.chunk], np.int32), H, w.scale, dt)
+        assert gh.max_excess(out[sl], ref, dt) <= gh.TOL[dt], s

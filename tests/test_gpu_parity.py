@@ -407,7 +407,7 @@ def test_prefill_matches_oracle(hq, hkv, d, dtype):
     qchunk = wl.draw_values(rng, (int(qlens.sum()), hq, d), dtype)
     out, ref = run_prefill(p, qchunk, qlens)
     assert pk.get_error() == (0, 0)
-    assert gh.max_err(out, ref) <= gh.TOL[dtype]
+    assert gh.max_excess(out, ref, dtype) <= gh.TOL[dtype]
 
 
 def test_prefill_one_token_chunks_agree_with_decode():
@@ -416,7 +416,7 @@ def test_prefill_one_token_chunks_agree_with_decode():
     p = make_paged(rng, 4, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
     out, ref = run_prefill(p, p.q, np.ones(4, np.int32))
     dec = gpu_out(p)
-    assert gh.max_err(out, ref) <= gh.TOL[wl.BF16]
+    assert gh.max_excess(out, ref, wl.BF16) <= gh.TOL[wl.BF16]
     assert float((out.float() - dec.float()).abs().max()) <= gh.TOL[wl.BF16]
 
 
@@ -429,7 +429,7 @@ def test_prefill_long_contexts_and_slack_grid():
     p = make_paged(rng, 3, 32, 8, 128, lens, wl.blocks_needed(lens, 16) + 1, wl.BF16)
     qchunk = wl.draw_values(rng, (int(qlens.sum()), 32, 128), wl.BF16)
     out, ref = run_prefill(p, qchunk, qlens, max_query_len=900)
-    assert gh.max_err(out, ref) <= gh.TOL[wl.BF16]
+    assert gh.max_excess(out, ref, wl.BF16) <= gh.TOL[wl.BF16]
 
 
 def test_prefill_chunk_longer_than_context_is_reported():
@@ -447,7 +447,7 @@ def test_prefill_chunk_longer_than_context_is_reported():
     assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_CONTEXT_LEN
     ref = oracle.prefill(qchunk[25:], p.key_cache, p.value_cache, p.tables[1:], p.lens[1:],
                          np.array([0, 30], np.int32), 4, p.scale, wl.F16)
-    assert gh.max_err(out[25:], ref) <= gh.TOL[wl.F16]
+    assert gh.max_excess(out[25:], ref, wl.F16) <= gh.TOL[wl.F16]
 
 
 # ---------------------------------------------------------------- CUDA graph capture
