@@ -7,6 +7,7 @@
 #include <cstring>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "pa_api.h"
 #include "pa_kernels.cuh"
@@ -104,10 +105,26 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
                : PA_ERR_CUDA;
 }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` (once per kernel,
+// device and size: the attribute persists in the context).
 template <typename Kernel>
 bool set_smem(Kernel k, int bytes) {
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-           cudaSuccess;
+    struct Key {
+        const void *fn;
+        int dev, bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Key> done;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const void *fn = reinterpret_cast<const void *>(k);
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Key &e : done)
+        if (e.fn == fn && e.dev == dev && e.bytes >= bytes) return true;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    done.push_back({fn, dev, bytes});
+    return true;
 }
 
 template <typename T, int D>
