@@ -286,6 +286,16 @@ int pa_swap_blocks(const void *src_key_cache, const void *src_value_cache, int64
  */
 int pa_get_error(void *stream, uint32_t *bits);
 
+/*
+ * pa_selftest_wait_timeout - diagnostic of the failure path shared by every
+ * kernel: one warp waits on an mbarrier that nothing completes, gives up
+ * after timeout_ns (1 ns .. 1 s) and sets PA_DEVERR_TIMEOUT, exactly as a
+ * decode or prefill CTA does when a TMA tile never lands.  A following
+ * pa_get_error returns PA_ERR_TIMEOUT; the CUDA context stays usable.  It has
+ * no counterpart in the pages.
+ */
+int pa_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
+
 /* Static description of a status code. */
 const char *pa_status_string(int status);
 

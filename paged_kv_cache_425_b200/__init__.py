@@ -86,6 +86,7 @@ pa_copy_blocks = _sig("pa_copy_blocks", ctypes.c_int, _P, _P, _P, _i32, _i32, _i
 pa_swap_blocks = _sig("pa_swap_blocks", ctypes.c_int, _P, _P, _i64, _P, _P, _i64, _P, _i32, _i32,
                       _i32, _i32, _i32, _P)
 pa_get_error = _sig("pa_get_error", ctypes.c_int, _P, ctypes.POINTER(ctypes.c_uint32))
+pa_selftest_wait_timeout = _sig("pa_selftest_wait_timeout", ctypes.c_int, ctypes.c_uint64, _P)
 pa_status_string = _sig("pa_status_string", ctypes.c_char_p, ctypes.c_int)
 pa_version = _sig("pa_version", ctypes.c_int)
 pa_alloc_create = _sig("pa_alloc_create", _P, _i32, _i32)
@@ -287,6 +288,11 @@ def swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, 
                           ctypes.c_void_p(dst_value_cache.data_ptr()), dnb,
                           pairs.ctypes.data if len(pairs) else None, int(len(pairs)), hkv, d, bs,
                           dtype_code(src_key_cache), _stream(stream)), "pa_swap_blocks")
+
+
+def selftest_wait_timeout(timeout_ns: int = 1_000_000, stream=None):
+    """Run the bounded-wait failure path once on the device (see pa_api.h)."""
+    _check(pa_selftest_wait_timeout(int(timeout_ns), _stream(stream)), "pa_selftest_wait_timeout")
 
 
 def get_error(stream=None):

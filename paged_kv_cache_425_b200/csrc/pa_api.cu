@@ -455,6 +455,12 @@ int pa_get_error(void *stream, uint32_t *bits) {
     return (word & PA_DEVERR_TIMEOUT) ? PA_ERR_TIMEOUT : PA_ERR_OUT_OF_RANGE;
 }
 
+int pa_selftest_wait_timeout(uint64_t timeout_ns, void *stream) {
+    if (timeout_ns == 0 || timeout_ns > 1000000000ull) return PA_ERR_INVALID_ARG;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 const char *pa_status_string(int status) {
     switch (status) {
         case PA_OK: return "ok";

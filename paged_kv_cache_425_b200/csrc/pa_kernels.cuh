@@ -1044,4 +1044,18 @@ __global__ void swap_blocks_kernel(const uint4 *__restrict__ sk, const uint4 *__
     }
 }
 
+// ------------------------------------------------------------------ bounded-wait self test
+// One warp waits on a fresh mbarrier that nothing will ever complete, through
+// the same bounded wait every kernel above uses; after timeout_ns it records
+// PA_DEVERR_TIMEOUT and returns.
+__global__ void wait_selftest_kernel(unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    mbar_wait_bounded(&bar, 0, timeout_ns);
+}
+
 }  // namespace pa

@@ -487,3 +487,18 @@ def test_decode_step_replays_from_a_cuda_graph():
         torch.cuda.synchronize()
         assert torch.equal(out, eager)
     assert pk.get_error() == (0, 0)
+
+
+# ---------------------------------------------------------------- bounded waits
+def test_a_wait_that_never_completes_times_out_and_the_context_survives():
+    """The bounded mbarrier wait every kernel uses gives up (1 ms here), sets
+    the timeout bit, and leaves the context usable for the next call."""
+    assert pk.get_error() == (0, 0)
+    pk.selftest_wait_timeout(1_000_000)
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_TIMEOUT and bits == pk.DEVERR_TIMEOUT
+    assert pk.get_error() == (0, 0)
+    rng = wl.rng_for(60)
+    lens = np.array([600, 20], np.int32)
+    p = make_paged(rng, 2, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
+    assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[wl.BF16]
