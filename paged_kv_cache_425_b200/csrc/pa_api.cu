@@ -324,6 +324,7 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
         return PA_ERR_UNSUPPORTED;
     constexpr int STAGES = 4;
     const size_t smem = (size_t)STAGES * 2 * kBlock * head_dim * 2 + 1024 +
+                        (size_t)(head_dim == 128 ? prefill_q_bytes<128>() : prefill_q_bytes<64>()) +
                         (size_t)max_blocks_per_seq * 4;
     if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
     PrefillArgs a;

@@ -744,8 +744,13 @@ struct PrefillArgs {
 
 constexpr float kMaskedLogit = -1.0e30f;  // finite, so 2^(masked - max) is exactly 0
 
+// Shared memory of one prefill CTA beyond its TMA ring: the 64 query rows,
+// each padded by 16 bytes so ldmatrix rows fall in different banks.
+template <int D>
+constexpr int prefill_q_bytes() { return 64 * (D * 2 + 16); }
+
 template <typename T, int D, int STAGES>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 4)
     prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const PrefillArgs a) {
     constexpr int NW = 4, ROWS = 64, KS = D / 16, NTD = D / 8;
@@ -753,8 +758,10 @@ __global__ void __launch_bounds__(128)
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t full_bar[STAGES];
     __shared__ __align__(8) uint64_t empty_bar[STAGES];
+    constexpr int QSTRIDE = D * 2 + 16;  // bytes per query row in shared memory
     uint8_t *ring = align_smem_1024(dyn_smem);
-    int32_t *s_table = reinterpret_cast<int32_t *>(ring + STAGES * STAGE);
+    uint8_t *s_q = ring + STAGES * STAGE;
+    int32_t *s_table = reinterpret_cast<int32_t *>(s_q + prefill_q_bytes<D>());
 
     const int G = a.num_q_heads / a.num_kv_heads;
     const int s = blockIdx.x / a.num_kv_heads, kvh = blockIdx.x % a.num_kv_heads;
@@ -836,16 +843,25 @@ __global__ void __launch_bounds__(128)
     }
     const int wlast = min(rbase + 15, rows_total - 1);
     const int warp_pmax = wlast >= rbase ? L - n + wlast / G : -1;
-    // A operand (Q rows) for all k-steps
-    uint32_t qa[KS][4];
-    const uint16_t *qb = reinterpret_cast<const uint16_t *>(a.q);
-#pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-        qa[kk][0] = rvalid[0] ? *reinterpret_cast<const uint32_t *>(qb + qrow[0] + 16 * kk + 2 * c) : 0u;
-        qa[kk][1] = rvalid[1] ? *reinterpret_cast<const uint32_t *>(qb + qrow[1] + 16 * kk + 2 * c) : 0u;
-        qa[kk][2] = rvalid[0] ? *reinterpret_cast<const uint32_t *>(qb + qrow[0] + 16 * kk + 8 + 2 * c) : 0u;
-        qa[kk][3] = rvalid[1] ? *reinterpret_cast<const uint32_t *>(qb + qrow[1] + 16 * kk + 8 + 2 * c) : 0u;
+    // the CTA's 64 query rows into shared memory (zero rows past the chunk);
+    // each warp reads its A fragments from there with ldmatrix per k-step
+    {
+        const uint4 *qg = reinterpret_cast<const uint4 *>(a.q);
+        for (int idx = tid; idx < ROWS * (D / 8); idx += NW * 32) {
+            const int r = idx / (D / 8), ch = idx % (D / 8);
+            const int R = tile * ROWS + r;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (R < rows_total) {
+                const size_t row = (size_t)(q0 + R / G) * a.num_q_heads + (size_t)kvh * G + R % G;
+                v = qg[row * (D / 8) + ch];
+            }
+            *reinterpret_cast<uint4 *>(s_q + r * QSTRIDE + ch * 16) = v;
+        }
     }
+    __syncthreads();
+    const uint32_t q_frag_base =
+        smem_addr(s_q) + (uint32_t)((warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * QSTRIDE +
+                                    (lane >> 4) * 16);
     float o[NTD][4];
 #pragma unroll
     for (int j = 0; j < NTD; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -884,13 +900,15 @@ __global__ void __launch_bounds__(128)
             for (int t = 0; t < 4; ++t) sf[t][0] = sf[t][1] = sf[t][2] = sf[t][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
+                uint32_t qa[4];
+                ldmatrix_x4(qa, q_frag_base + kk * 32);
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
                     if (!use[bb]) continue;
                     uint32_t b[4];
                     ldmatrix_x4(b, kt[bb] + tile_off(k_row, 2 * kk + k_half));
-                    Mma<T>::run(sf[2 * bb], qa[kk], b[0], b[1]);
-                    Mma<T>::run(sf[2 * bb + 1], qa[kk], b[2], b[3]);
+                    Mma<T>::run(sf[2 * bb], qa, b[0], b[1]);
+                    Mma<T>::run(sf[2 * bb + 1], qa, b[2], b[3]);
                 }
             }
             float pv[4][4], alpha_row[2];
