@@ -83,18 +83,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // ---------------------------------------------------------------- TMA
-// 2-D tiled tensor load of box (x, y) into shared memory, completing
-// `bytes` of transaction count on `bar`.  x must be a multiple of 16 bytes.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
-                                            int32_t x, int32_t y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-
-// Same, with an L2 eviction-priority hint (streamed data: evict first).
+// 2-D tiled tensor load of box (x, y) into shared memory, completing its
+// bytes of transaction count on `bar`, with an L2 eviction-priority hint
+// (streamed data: evict first).  x * element size must be a multiple of 16.
 __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map,
                                                  uint64_t *bar, int32_t x, int32_t y,
                                                  uint64_t policy) {
@@ -109,10 +100,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
-}
-
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // ---------------------------------------------------------------- fragments
@@ -178,12 +165,6 @@ __device__ __forceinline__ float2 widen2(uint32_t bits, __half) {
 __device__ __forceinline__ float2 widen2(uint32_t bits, __nv_bfloat16) {
     // bf16 -> f32 is exact: the bf16 bits are the top half of the f32.
     return make_float2(__uint_as_float(bits << 16), __uint_as_float(bits & 0xffff0000u));
-}
-__device__ __forceinline__ float widen1(uint16_t bits, __half) {
-    return __half2float(__ushort_as_half(bits));
-}
-__device__ __forceinline__ float widen1(uint16_t bits, __nv_bfloat16) {
-    return __uint_as_float(static_cast<uint32_t>(bits) << 16);
 }
 __device__ __forceinline__ uint16_t narrow1(float x, __half) {
     return __half_as_ushort(__float2half_rn(x));

@@ -169,12 +169,6 @@ struct WarpPipe {
     }
 };
 
-// Common prologue of both decode kernels.  Returns false if this CTA has no
-// partition to process (it may still have written a zero row).
-struct PartitionInfo {
-    int L, nblk, nparts, b_begin, nk;
-};
-
 __device__ __forceinline__ int warp_block_count(int nb_local, int warp, int nw) {
     return warp < nb_local ? (nb_local - warp + nw - 1) / nw : 0;
 }
