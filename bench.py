@@ -49,7 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b",
-                    choices=["llama7b", "llama13b", "gqa_long", "cow", "tiny", "swap", "prefill"])
+                    choices=["llama7b", "llama13b", "gqa_long", "cow", "cow_run", "tiny", "swap",
+                             "prefill"])
     ap.add_argument("--layers", type=int, default=0,
                     help="layer caches to allocate (0: the workload's layer count; fewer "
                          "caches are cycled so every step still runs every layer)")
@@ -326,16 +327,16 @@ def run_ours(args, world, rank, local):
     barrier(device)
     torch.cuda.synchronize()
     sampler.start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(st.stream)
-    for _ in range(args.steps):
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    marks[0].record(st.stream)
+    for i in range(args.steps):
         st.step()
-    t1.record(st.stream)
+        marks[i + 1].record(st.stream)  # at step boundaries only
     torch.cuda.synchronize()
     barrier(device)
     clocks = sampler.stop()
-    local_ms = t0.elapsed_time(t1)
+    local_ms = marks[0].elapsed_time(marks[-1])
+    step_ms = [marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)]
     rc, bits = st.pk.get_error(st.stream)
     if rc != 0:
         raise RuntimeError(f"device error word {bits:#x} in the timed region")
@@ -379,6 +380,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4),
+        "ms_per_step_p10_p50_p90": [round(float(np.percentile(step_ms, q)), 4) for q in (10, 50, 90)],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -604,6 +606,117 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_cow_run(args, world, rank, local):
+    """The whole parallel-sampling run: every generation step of the 32 x 4
+    branches (step 0 copies the diverging shared last prompt block; later
+    steps decode a shrinking set of live branches), 32 layers per step.  All
+    steps' tables, lengths, slots and copy pairs come from the allocator
+    before timing; the run is captured once in a CUDA graph and replayed, so
+    host launch overhead stays out of the timing.  value = mean tokens/s."""
+    import torch
+    import paged_kv_cache_425_b200 as pk
+    from paged_kv_cache_425_b200 import batch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    w = wl.WORKLOADS["cow"]
+    rng = wl.rng_for(args.seed + rank)
+    own = wl.draw_branch_tokens(w, rng)
+    nb = batch.cow_pool_blocks(w)
+    fb = batch.ForkedBatch(w, own, wl.draw_block_order(nb, rng), nb)
+    plan = []
+    while fb.step_index < fb.num_steps:
+        b = fb.step()
+        plan.append((torch.from_numpy(b.tables).to(device), torch.from_numpy(b.context_lens).to(device),
+                     torch.from_numpy(b.slots).to(device),
+                     torch.from_numpy(b.pairs).to(device) if len(b.pairs) else None,
+                     len(b.seq_ids), algorithmic_bytes(b.context_lens, w.num_q_heads, w.num_kv_heads,
+                                                       w.head_dim)))
+    tokens_per_run = sum(p[4] for p in plan)
+    bytes_per_run = sum(p[5] for p in plan) * w.layers
+    S, H, Hq, d, L = w.num_seqs, w.num_kv_heads, w.num_q_heads, w.head_dim, w.layers
+    ncache = min(args.layers if args.layers > 0 else L, L)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(3000 + args.seed + rank)
+    kc = [torch.randn((nb, H, 16, d), generator=gen, device=device, dtype=torch.bfloat16)
+          for _ in range(ncache)]
+    vc = [torch.randn((nb, H, 16, d), generator=gen, device=device, dtype=torch.bfloat16)
+          for _ in range(ncache)]
+    q = torch.randn((L, S, Hq, d), generator=gen, device=device, dtype=torch.bfloat16)
+    kn = torch.randn((L, S, H, d), generator=gen, device=device, dtype=torch.bfloat16)
+    vn = torch.randn((L, S, H, d), generator=gen, device=device, dtype=torch.bfloat16)
+    out = torch.empty_like(q)
+    nws = pk.decode_workspace_size(S, Hq, d, fb.max_blocks)
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=device)
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.Stream(device)
+
+    def run():
+        for tables, lens, slots, pairs, n, _ in plan:
+            for l in range(L):
+                c = l % ncache
+                if pairs is not None:
+                    pk.copy_blocks(kc[c], vc[c], pairs, stream=stream)
+                pk.reshape_and_cache(kn[l][:n], vn[l][:n], kc[c], vc[c], slots, stream=stream)
+                pk.decode(out[l][:n], q[l][:n], kc[c], vc[c], tables, lens, H, w.scale,
+                          workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    for _ in range(args.warmup):
+        graph.replay()
+    rc, bits = pk.get_error()
+    if rc != 0:
+        raise RuntimeError(f"device error word {bits:#x}")
+    sampler = ClockSampler(device)
+    barrier(device)
+    torch.cuda.synchronize()
+    sampler.start()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream(device)
+    a.record(cur)
+    for _ in range(args.steps):
+        graph.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    barrier(device)
+    clocks = sampler.stop()
+    ms = max_over_ranks(a.elapsed_time(b), device)
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    per_run_s = ms * 1e-3 / args.steps
+    peak, src = load_peak()
+    gbs = bytes_per_run / per_run_s / 1e9
+    print(json.dumps({
+        "metric": "parallel-sampling run: mean decode tokens/s over the whole generation",
+        "value": round(world * tokens_per_run / per_run_s, 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_run": round(per_run_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "cow_run: 32 prompts x 4 branches, 1000-token prompt, branch b "
+                               "generates 1 + U{0..256} tokens, 32 layers per step",
+                   "generation_steps": len(plan), "tokens_per_run": tokens_per_run,
+                   "layer_caches": ncache, "timing": "whole run captured in one CUDA graph"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "kernel": "whole run (copy + scatter + decode), logical bytes",
+                     "peak_source": src},
+        "gpu_launches": args.steps * sum(L * (2 + (1 if p[3] is not None else 0) + 1)
+                                         for p in plan),
+        "clocks": clocks}), flush=True)
+
+
 def prefill_flops(lens, chunk, num_q_heads, head_dim):
     """Multiply-adds x 2 of chunked prefill: query token i of a sequence with
     context L attends to L - chunk + i + 1 keys, for q.K and for P.V."""
@@ -785,10 +898,13 @@ def main(argv=None):
     if args.workload == "prefill" and args.impl == "ours":
         run_prefill(args, world, rank, local)
         return 0
+    if args.workload == "cow_run" and args.impl == "ours":
+        run_cow_run(args, world, rank, local)
+        return 0
     if world > 1 and args.gpus != world:
         args.gpus = world
     if args.impl == "reference":
-        if args.workload in ("swap", "prefill"):
+        if args.workload in ("swap", "prefill", "cow_run"):
             if rank == 0:
                 print(json.dumps({"impl": "reference", "unavailable":
                                   "the CPU reference arm times decode workloads only"}))
