@@ -188,7 +188,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
 /*
  * pa_decode_static_workspace - pa_decode for callers that cannot allocate.
  *
- * The pages have no counterpart for this call: it is an interface
+ * The paper has no counterpart for this call: it is an interface
  * convenience of this library, not a step of the method.
  *
  * pa_decode needs split-context scratch (its `workspace`) whenever a context
