@@ -415,7 +415,8 @@ def run_e2e(st, args, device, world, chunks: int = 4):
     inputs of the next group of layers while the current group computes, and
     reads each group's outputs back as soon as they are done; per-group events
     keep a step's copies from overwriting buffers the previous step still
-    uses."""
+    uses, so one step's last read-back overlaps the next step's compute.  The
+    region ends once the last step's outputs are on the host."""
     import torch
     L = st.layers
     per = (L + chunks - 1) // chunks
@@ -477,14 +478,19 @@ def run_e2e(st, args, device, world, chunks: int = 4):
                 copy.wait_event(ev_done[c])
                 hout[a:b].copy_(st.out[a:b], non_blocking=True)
                 ev_read[c].record(copy)
-        comp.wait_event(ev_read[-1])                  # the step ends when its outputs are back
         first[0] = False
 
     # with one layer group there is nothing to overlap: one stream, no syncs
     one = one_overlapped if len(groups) > 1 else one_serial
 
+    def drain():
+        # the timed region ends when the last outputs are back on the host
+        if one is one_overlapped:
+            comp.wait_event(ev_read[-1])
+
     for _ in range(max(1, args.warmup)):
         one()
+    drain()
     barrier(device)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
@@ -492,6 +498,7 @@ def run_e2e(st, args, device, world, chunks: int = 4):
     a.record(comp)
     for _ in range(args.steps):
         one()
+    drain()
     b.record(comp)
     torch.cuda.synchronize()
     barrier(device)
