@@ -57,6 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="run the workload with fewer sequences (small profiling case; "
                          "the bench line then names the reduced size)")
+    ap.add_argument("--prefill-kernel", choices=["auto", "mma_sync", "tcgen05"], default="auto",
+                    help="prefill workload: which pa_prefill kernel runs (auto = tcgen05)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -781,6 +783,9 @@ def run_prefill(args, world, rank, local):
     d_slots = torch.from_numpy(np.concatenate(slots)).to(device)
     torch.cuda.synchronize(device)
     stream = torch.cuda.Stream(device)
+    pk.prefill_select(args.prefill_kernel)
+    kernel_name = ("prefill_mma_kernel (mma.sync m16n8k16)" if args.prefill_kernel == "mma_sync"
+                   else "prefill_umma_kernel (tcgen05.mma, TMEM accumulators)")
 
     def step():
         for l in range(layers):
@@ -843,7 +848,7 @@ def run_prefill(args, world, rank, local):
         "config": {**describe(w, ctx, ncache), "chunk": chunk, "query_tokens_per_step_layer": T},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
-                     "kernel": "prefill_mma_kernel (mma.sync m16n8k16)", "flops_per_call": flops,
+                     "kernel": kernel_name, "flops_per_call": flops,
                      "avg_call_us": round(call_ms * 1e3, 2), "peak_source": src},
         "gpu_launches": args.steps * layers * 2,
         "clocks": clocks,

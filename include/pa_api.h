@@ -180,6 +180,25 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
                int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
                int64_t num_blocks, int32_t dtype, void *stream);
 
+/*
+ * pa_prefill_select - which kernel pa_prefill runs (process-wide).
+ *
+ *   PA_PREFILL_AUTO     the tcgen05 kernel when its conditions hold (q and
+ *                       out 16-byte aligned, query group <= 128), otherwise
+ *                       the mma.sync kernel.  The default.
+ *   PA_PREFILL_MMA_SYNC always the mma.sync kernel (64 packed query rows per
+ *                       CTA, warp-level tensor-core tiles, registers hold S).
+ *   PA_PREFILL_TCGEN05  always the tcgen05 kernel (128 packed query rows per
+ *                       CTA, accumulators in tensor memory); pa_prefill
+ *                       returns PA_ERR_UNSUPPORTED when its conditions fail.
+ * Both compute the same operation; results differ only by rounding order.
+ * Returns PA_OK, or PA_ERR_INVALID_ARG for an unknown value.
+ */
+#define PA_PREFILL_AUTO 0
+#define PA_PREFILL_MMA_SYNC 1
+#define PA_PREFILL_TCGEN05 2
+int pa_prefill_select(int32_t kernel);
+
 /* Bytes of workspace pa_decode needs for these sizes (0 when no context can
  * exceed one partition). */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,

@@ -81,6 +81,7 @@ pa_decode_static_workspace = _sig("pa_decode_static_workspace", ctypes.c_int, _P
                                   _P, _i32, _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
 pa_prefill = _sig("pa_prefill", ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _f32, _i32,
                   _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
+pa_prefill_select = _sig("pa_prefill_select", ctypes.c_int, _i32)
 pa_copy_blocks = _sig("pa_copy_blocks", ctypes.c_int, _P, _P, _P, _i32, _i32, _i32, _i32, _i64,
                       _i32, _P)
 pa_swap_blocks = _sig("pa_swap_blocks", ctypes.c_int, _P, _P, _i64, _P, _P, _i64, _P, _i32, _i32,
@@ -230,6 +231,18 @@ def prefill(out, q, key_cache, value_cache, block_tables, context_lens, query_st
                       _dev(query_start, "query_start", torch.int32, 1), int(max_query_len), hkv,
                       float(scale), S, hq, T, d, bs, int(block_tables.shape[1]), nb, dtype_code(q),
                       _stream(stream)), "pa_prefill")
+
+
+PREFILL_KERNELS = {"auto": 0, "mma_sync": 1, "tcgen05": 2}
+
+
+def prefill_select(kernel: str) -> None:
+    """Which kernel prefill() runs, process-wide: "auto" (the tcgen05 kernel
+    when q / out are 16-byte aligned and the query group is at most 128, else
+    the mma.sync kernel), "mma_sync" or "tcgen05"."""
+    if kernel not in PREFILL_KERNELS:
+        raise ValueError(f"kernel must be one of {sorted(PREFILL_KERNELS)}")
+    _check(pa_prefill_select(PREFILL_KERNELS[kernel]), "pa_prefill_select")
 
 
 def decode_static_workspace(out, q, key_cache, value_cache, block_tables, context_lens,

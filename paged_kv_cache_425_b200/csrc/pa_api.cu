@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -11,6 +12,7 @@
 
 #include "pa_api.h"
 #include "pa_kernels.cuh"
+#include "pa_prefill_umma.cuh"
 
 namespace pa {
 namespace {
@@ -71,7 +73,32 @@ bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, i
     return r == CUDA_SUCCESS;
 }
 
+// TMA descriptor of the query rows of one kv head's group, viewed as 4-D:
+// (head_dim, G heads of the group, kv head, token), box = 64 columns x G x 1 x
+// TT tokens, so a box lands as TT * G rows of 128 bytes in packed-row order
+// (token i, head h -> row i * G + h); 128-byte swizzle; rows past the last
+// token read as zero.
+bool encode_q_map(CUtensorMap *map, const void *q, int num_q_tokens, int num_q_heads,
+                  int num_kv_heads, int head_dim, int dtype, int tokens_per_box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int G = num_q_heads / num_kv_heads;
+    cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)G, (cuuint64_t)num_kv_heads,
+                          (cuuint64_t)num_q_tokens};
+    cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)G * head_dim * 2,
+                             (cuuint64_t)num_q_heads * head_dim * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)tokens_per_box};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    4, const_cast<void *>(q), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+std::atomic<int> g_prefill_kernel{PA_PREFILL_AUTO};
 
 int check_cache_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                       int64_t num_blocks, int32_t dtype) {
@@ -204,6 +231,51 @@ WorkspaceLayout workspace_layout(int64_t num_seqs, int64_t num_q_heads, int64_t 
     return l;
 }
 
+// pa_prefill on the tcgen05 kernel: grid x = (sequence, kv head), y = tile of
+// 128 packed query rows (the largest multiple of the group size <= 128).
+int launch_prefill_umma(void *out, const void *q, const void *key_cache, const void *value_cache,
+                        const int32_t *block_tables, const int32_t *context_lens,
+                        const int32_t *query_start, int32_t max_query_len, int32_t num_kv_heads,
+                        float scale, int32_t num_seqs, int32_t num_q_heads, int32_t num_q_tokens,
+                        int32_t head_dim, int32_t max_blocks_per_seq, int64_t num_blocks,
+                        int32_t dtype, cudaStream_t st) {
+    const int group = num_q_heads / num_kv_heads;
+    const int tokens_per_tile = kUmmaRows / group;
+    const int64_t tiles = ((int64_t)max_query_len * group + tokens_per_tile * group - 1) /
+                          (tokens_per_tile * group);
+    PrefillArgs a;
+    a.out = out;
+    a.q = q;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.query_start = query_start;
+    a.num_blocks = num_blocks;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_q_tokens = num_q_tokens;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    CUtensorMap tmq, tmk, tmv;
+    if (!encode_q_map(&tmq, q, num_q_tokens, num_q_heads, num_kv_heads, head_dim, dtype,
+                      tokens_per_tile) ||
+        !encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
+        !encode_cache_map(&tmv, value_cache, num_blocks, num_kv_heads, head_dim, dtype))
+        return PA_ERR_CUDA;
+    const dim3 grid(num_seqs * num_kv_heads, (unsigned)tiles);
+    auto launch = [&](auto kernel, int smem) -> int {
+        if (!set_smem(kernel, smem)) return PA_ERR_CUDA;
+        return launch_pdl(kernel, grid, dim3(kUmmaThreads), (size_t)smem, st, tmq, tmk, tmv, a);
+    };
+    if (dtype == PA_F16)
+        return head_dim == 128
+                   ? launch(prefill_umma_kernel<__half, 128>, prefill_umma_smem_bytes<128>())
+                   : launch(prefill_umma_kernel<__half, 64>, prefill_umma_smem_bytes<64>());
+    return head_dim == 128
+               ? launch(prefill_umma_kernel<__nv_bfloat16, 128>, prefill_umma_smem_bytes<128>())
+               : launch(prefill_umma_kernel<__nv_bfloat16, 64>, prefill_umma_smem_bytes<64>());
+}
+
 }  // namespace
 }  // namespace pa
 
@@ -298,6 +370,13 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
                            : dispatch_decode<__nv_bfloat16>(a, head_dim, group, tmk, tmv, st);
 }
 
+int pa_prefill_select(int32_t kernel) {
+    if (kernel != PA_PREFILL_AUTO && kernel != PA_PREFILL_MMA_SYNC && kernel != PA_PREFILL_TCGEN05)
+        return PA_ERR_INVALID_ARG;
+    g_prefill_kernel.store(kernel);
+    return PA_OK;
+}
+
 int pa_prefill(void *out, const void *q, const void *key_cache, const void *value_cache,
                const int32_t *block_tables, const int32_t *context_lens,
                const int32_t *query_start, int32_t max_query_len, int32_t num_kv_heads,
@@ -319,9 +398,18 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
         !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(context_lens, 4) ||
         !aligned(query_start, 4))
         return PA_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs * num_kv_heads >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    const int which = g_prefill_kernel.load();
+    const bool umma_ok = group <= kUmmaRows && aligned(q, 16) && aligned(out, 16) &&
+                         (int64_t)max_query_len * group <= (int64_t)65535 * ((kUmmaRows / group) * group);
+    if (which == PA_PREFILL_TCGEN05 && !umma_ok) return PA_ERR_UNSUPPORTED;
+    if (which != PA_PREFILL_MMA_SYNC && umma_ok)
+        return launch_prefill_umma(out, q, key_cache, value_cache, block_tables, context_lens,
+                                   query_start, max_query_len, num_kv_heads, scale, num_seqs,
+                                   num_q_heads, num_q_tokens, head_dim, max_blocks_per_seq,
+                                   num_blocks, dtype, static_cast<cudaStream_t>(stream));
     const int64_t tiles = ((int64_t)max_query_len * group + 63) / 64;
-    if (tiles > 65535 || (int64_t)num_seqs * num_kv_heads >= (int64_t(1) << 31))
-        return PA_ERR_UNSUPPORTED;
+    if (tiles > 65535) return PA_ERR_UNSUPPORTED;
     constexpr int STAGES = 4;
     const size_t smem = (size_t)STAGES * 2 * kBlock * head_dim * 2 + 1024 +
                         (size_t)(head_dim == 128 ? prefill_q_bytes<128>() : prefill_q_bytes<64>()) +

@@ -434,3 +434,12 @@ def test_requests_larger_than_the_pool_are_rejected():
     st = pk.simulate_continuous_batching(10, 4, np.array([100, 400], np.int32),
                                          np.array([10, 10], np.int32))
     assert st["rejected"] == 1 and st["finished"] == 1
+
+
+def test_prefill_select_accepts_the_three_kernels_only():
+    assert pk.pa_prefill_select(7) == pk.PA_ERR_INVALID_ARG
+    assert pk.pa_prefill_select(-1) == pk.PA_ERR_INVALID_ARG
+    for name in ("mma_sync", "tcgen05", "auto"):
+        pk.prefill_select(name)
+    with pytest.raises(ValueError):
+        pk.prefill_select("wgmma")

@@ -381,12 +381,36 @@ def test_swap_out_and_back_in_is_bit_exact_and_decode_follows(pinned):
 
 
 # ---------------------------------------------------------------- chunked prefill
-def run_prefill(p, qchunk, qlens, max_query_len=None):
+@pytest.fixture(params=["mma_sync", "tcgen05"])
+def prefill_kernel(request):
+    """Run the test on each prefill kernel, then restore the default."""
+    pk.prefill_select(request.param)
+    yield request.param
+    pk.prefill_select("auto")
+
+
+def poisoned(p):
+    """Copies of p's pools with every row that holds no token of any
+    sequence (unused blocks, tails of last blocks) set to NaN."""
+    live = np.zeros(p.key_cache.shape[:1] + p.key_cache.shape[2:3], bool)  # [block, slot]
+    for s, L in enumerate(p.lens):
+        for t in range(int(L)):
+            live[p.tables[s, t // 16], t % 16] = True
+    nan = np.uint16(0x7E00 if p.dtype == wl.F16 else 0x7FC0)
+    kc, vc = p.key_cache.copy(), p.value_cache.copy()
+    dead = ~live
+    kc.transpose(0, 2, 1, 3)[dead] = nan
+    vc.transpose(0, 2, 1, 3)[dead] = nan
+    return kc, vc
+
+
+def run_prefill(p, qchunk, qlens, max_query_len=None, pools=None):
     qs = np.zeros(len(qlens) + 1, np.int32)
     qs[1:] = np.cumsum(qlens)
     q = gh.to_dev(qchunk, p.dtype)
     out = torch.full_like(q, float("nan"))
-    pk.prefill(out, q, gh.to_dev(p.key_cache, p.dtype), gh.to_dev(p.value_cache, p.dtype),
+    kc, vc = pools if pools is not None else (p.key_cache, p.value_cache)
+    pk.prefill(out, q, gh.to_dev(kc, p.dtype), gh.to_dev(vc, p.dtype),
                gh.ints(p.tables), gh.ints(p.lens), gh.ints(qs),
                int(max(qlens)) if max_query_len is None else max_query_len, p.num_kv_heads,
                p.scale)
@@ -399,7 +423,7 @@ def run_prefill(p, qchunk, qlens, max_query_len=None):
 @pytest.mark.parametrize("hq,hkv,d,dtype", [(4, 4, 64, wl.F16), (8, 2, 128, wl.BF16),
                                             (32, 8, 128, wl.BF16), (8, 1, 64, wl.F16),
                                             (16, 16, 128, wl.F16)])
-def test_prefill_matches_oracle(hq, hkv, d, dtype):
+def test_prefill_matches_oracle(hq, hkv, d, dtype, prefill_kernel):
     rng = wl.rng_for(40 + hq + d)
     lens = np.array([40, 700, 17, 64, 5, 1, 513], np.int32)
     qlens = np.array([40, 300, 1, 16, 5, 1, 77], np.int32)  # whole prompts, chunks, single tokens
@@ -410,7 +434,7 @@ def test_prefill_matches_oracle(hq, hkv, d, dtype):
     assert gh.max_excess(out, ref, dtype) <= gh.TOL[dtype]
 
 
-def test_prefill_one_token_chunks_agree_with_decode():
+def test_prefill_one_token_chunks_agree_with_decode(prefill_kernel):
     rng = wl.rng_for(41)
     lens = np.array([33, 1, 1200, 512], np.int32)
     p = make_paged(rng, 4, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
@@ -420,7 +444,7 @@ def test_prefill_one_token_chunks_agree_with_decode():
     assert float((out.float() - dec.float()).abs().max()) <= gh.TOL[wl.BF16]
 
 
-def test_prefill_long_contexts_and_slack_grid():
+def test_prefill_long_contexts_and_slack_grid(prefill_kernel):
     """Chunks of 512 over contexts up to 4k, with a grid sized for a larger
     max_query_len than any sequence uses."""
     rng = wl.rng_for(42)
@@ -432,7 +456,7 @@ def test_prefill_long_contexts_and_slack_grid():
     assert gh.max_excess(out, ref, wl.BF16) <= gh.TOL[wl.BF16]
 
 
-def test_prefill_chunk_longer_than_context_is_reported():
+def test_prefill_chunk_longer_than_context_is_reported(prefill_kernel):
     rng = wl.rng_for(43)
     lens = np.array([20, 30], np.int32)
     p = make_paged(rng, 2, 4, 4, 64, lens, 4, wl.F16)
@@ -448,6 +472,89 @@ def test_prefill_chunk_longer_than_context_is_reported():
     ref = oracle.prefill(qchunk[25:], p.key_cache, p.value_cache, p.tables[1:], p.lens[1:],
                          np.array([0, 30], np.int32), 4, p.scale, wl.F16)
     assert gh.max_excess(out[25:], ref, wl.F16) <= gh.TOL[wl.F16]
+
+
+@pytest.mark.parametrize("hq,hkv", [(12, 4), (40, 8), (16, 1), (64, 2)])
+def test_prefill_groups_that_do_not_divide_the_tile(hq, hkv, prefill_kernel):
+    """Query groups of 3, 5, 16 and 32 heads: the tcgen05 tile holds the
+    largest multiple of the group that fits 128 rows (126, 125, 128, 128)."""
+    rng = wl.rng_for(44 + hq)
+    lens = np.array([300, 77, 1000], np.int32)
+    qlens = np.array([300, 50, 129], np.int32)
+    p = make_paged(rng, 3, hq, hkv, 128, lens, wl.blocks_needed(lens, 16) + 2, wl.BF16)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), hq, 128), wl.BF16)
+    out, ref = run_prefill(p, qchunk, qlens)
+    assert pk.get_error() == (0, 0)
+    assert gh.max_excess(out, ref, wl.BF16) <= gh.TOL[wl.BF16]
+
+
+@pytest.mark.parametrize("d,dtype", [(128, wl.BF16), (64, wl.F16)])
+def test_prefill_ignores_nan_in_rows_without_tokens(d, dtype, prefill_kernel):
+    """Every pool row that holds no token (unused blocks, the tail of each
+    last block) is NaN in K and V; the outputs must not see it."""
+    rng = wl.rng_for(45 + d)
+    lens = np.array([130, 17, 700, 1, 260], np.int32)
+    qlens = np.array([130, 3, 200, 1, 60], np.int32)
+    p = make_paged(rng, 5, 8, 2, d, lens, wl.blocks_needed(lens, 16) + 4, dtype)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), 8, d), dtype)
+    out, ref = run_prefill(p, qchunk, qlens, pools=poisoned(p))
+    assert pk.get_error() == (0, 0)
+    assert gh.max_excess(out, ref, dtype) <= gh.TOL[dtype]
+
+
+def test_prefill_bad_block_id_is_reported(prefill_kernel):
+    """An out-of-range id inside one sequence's range raises
+    PA_DEVERR_BLOCK_ID; the other sequences are still exact."""
+    rng = wl.rng_for(46)
+    lens = np.array([200, 300], np.int32)
+    qlens = np.array([64, 100], np.int32)
+    p = make_paged(rng, 2, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
+    p.tables[0, 3] = p.key_cache.shape[0] + 7
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), 8, 128), wl.BF16)
+    qs = np.array([0, 64, 164], np.int32)
+    q = gh.to_dev(qchunk, wl.BF16)
+    out = torch.zeros_like(q)
+    pk.prefill(out, q, gh.to_dev(p.key_cache, wl.BF16), gh.to_dev(p.value_cache, wl.BF16),
+               gh.ints(p.tables), gh.ints(p.lens), gh.ints(qs), 100, 2, p.scale)
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_BLOCK_ID
+    ref = oracle.prefill(qchunk[64:], p.key_cache, p.value_cache, p.tables[1:], p.lens[1:],
+                         np.array([0, 100], np.int32), 2, p.scale, wl.BF16)
+    assert gh.max_excess(out[64:], ref, wl.BF16) <= gh.TOL[wl.BF16]
+
+
+def test_prefill_kernels_agree():
+    """The two prefill kernels on one problem: both within the budget of
+    the oracle, and within twice that budget of each other."""
+    rng = wl.rng_for(47)
+    lens = np.array([2048, 900, 513], np.int32)
+    qlens = np.array([512, 512, 513], np.int32)
+    p = make_paged(rng, 3, 32, 8, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), 32, 128), wl.BF16)
+    outs = {}
+    try:
+        for k in ("mma_sync", "tcgen05"):
+            pk.prefill_select(k)
+            outs[k], ref = run_prefill(p, qchunk, qlens)
+            assert gh.max_excess(outs[k], ref, wl.BF16) <= gh.TOL[wl.BF16], k
+    finally:
+        pk.prefill_select("auto")
+    diff = (outs["mma_sync"].double() - outs["tcgen05"].double()).abs()
+    lim = 2 * (gh.TOL[wl.BF16] + gh.REL[wl.BF16] * torch.from_numpy(np.abs(ref)).cuda())
+    assert bool((diff <= lim).all())
+
+
+def test_decode_ignores_nan_in_rows_without_tokens():
+    """Decode on a pool whose token-free rows are NaN: every kernel (one
+    query head per kv head, grouped, split contexts) must not see it."""
+    for hq, hkv, dtype in ((8, 8, wl.F16), (16, 2, wl.BF16)):
+        rng = wl.rng_for(48 + hq)
+        lens = np.array([1, 17, 513, 1500, 33, 1024], np.int32)
+        p = make_paged(rng, 6, hq, hkv, 128, lens, wl.blocks_needed(lens, 16) + 5, dtype)
+        kc, vc = poisoned(p)
+        out = gh.run_decode(pk, p.q, kc, vc, p.tables, p.lens, hkv, p.scale, dtype)
+        assert pk.get_error() == (0, 0)
+        assert gh.max_err(out, oracle_out(p)) <= gh.TOL[dtype]
 
 
 # ---------------------------------------------------------------- CUDA graph capture
