@@ -241,8 +241,8 @@ int launch_prefill_umma(void *out, const void *q, const void *key_cache, const v
                         int32_t dtype, cudaStream_t st) {
     const int group = num_q_heads / num_kv_heads;
     const int tokens_per_tile = kUmmaRows / group;
-    const int64_t tiles = ((int64_t)max_query_len * group + tokens_per_tile * group - 1) /
-                          (tokens_per_tile * group);
+    const int64_t rows_per_cta = (int64_t)kUmmaQTiles * tokens_per_tile * group;
+    const int64_t tiles = ((int64_t)max_query_len * group + rows_per_cta - 1) / rows_per_cta;
     PrefillArgs a;
     a.out = out;
     a.q = q;
@@ -256,24 +256,33 @@ int launch_prefill_umma(void *out, const void *q, const void *key_cache, const v
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.num_q_tokens = num_q_tokens;
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.tiles_per_seq = (int)tiles;
     CUtensorMap tmq, tmk, tmv;
     if (!encode_q_map(&tmq, q, num_q_tokens, num_q_heads, num_kv_heads, head_dim, dtype,
                       tokens_per_tile) ||
         !encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
         !encode_cache_map(&tmv, value_cache, num_blocks, num_kv_heads, head_dim, dtype))
         return PA_ERR_CUDA;
-    const dim3 grid(num_seqs * num_kv_heads, (unsigned)tiles);
-    auto launch = [&](auto kernel, int smem) -> int {
+    const int64_t ctas = (int64_t)num_seqs * num_kv_heads * tiles;
+    if (ctas >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)ctas);
+    const int smem = head_dim == 128 ? prefill_umma_smem_bytes<128>(max_blocks_per_seq)
+                                     : prefill_umma_smem_bytes<64>(max_blocks_per_seq);
+    auto launch = [&](auto kernel) -> int {
+        // the kernel re-splits its registers per warpgroup (setmaxnreg); a
+        // split above what the launch holds would wait forever, so check the
+        // compiled count first
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return PA_ERR_CUDA;
+        if ((int64_t)fa.numRegs * kUmmaThreads < kUmmaRegsNeeded) return PA_ERR_UNSUPPORTED;
         if (!set_smem(kernel, smem)) return PA_ERR_CUDA;
         return launch_pdl(kernel, grid, dim3(kUmmaThreads), (size_t)smem, st, tmq, tmk, tmv, a);
     };
     if (dtype == PA_F16)
-        return head_dim == 128
-                   ? launch(prefill_umma_kernel<__half, 128>, prefill_umma_smem_bytes<128>())
-                   : launch(prefill_umma_kernel<__half, 64>, prefill_umma_smem_bytes<64>());
-    return head_dim == 128
-               ? launch(prefill_umma_kernel<__nv_bfloat16, 128>, prefill_umma_smem_bytes<128>())
-               : launch(prefill_umma_kernel<__nv_bfloat16, 64>, prefill_umma_smem_bytes<64>());
+        return head_dim == 128 ? launch(prefill_umma_kernel<__half, 128>)
+                               : launch(prefill_umma_kernel<__half, 64>);
+    return head_dim == 128 ? launch(prefill_umma_kernel<__nv_bfloat16, 128>)
+                           : launch(prefill_umma_kernel<__nv_bfloat16, 64>);
 }
 
 }  // namespace
@@ -400,14 +409,20 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
         return PA_ERR_INVALID_ARG;
     if ((int64_t)num_seqs * num_kv_heads >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
     const int which = g_prefill_kernel.load();
+    const int64_t umma_smem = (head_dim == 128 ? prefill_umma_smem_bytes<128>(0)
+                                               : prefill_umma_smem_bytes<64>(0)) +
+                              4 * (int64_t)max_blocks_per_seq;
     const bool umma_ok = group <= kUmmaRows && aligned(q, 16) && aligned(out, 16) &&
-                         (int64_t)max_query_len * group <= (int64_t)65535 * ((kUmmaRows / group) * group);
+                         scale > 0.f && scale < 3.0e38f && umma_smem <= 227 * 1024;
     if (which == PA_PREFILL_TCGEN05 && !umma_ok) return PA_ERR_UNSUPPORTED;
-    if (which != PA_PREFILL_MMA_SYNC && umma_ok)
-        return launch_prefill_umma(out, q, key_cache, value_cache, block_tables, context_lens,
-                                   query_start, max_query_len, num_kv_heads, scale, num_seqs,
-                                   num_q_heads, num_q_tokens, head_dim, max_blocks_per_seq,
-                                   num_blocks, dtype, static_cast<cudaStream_t>(stream));
+    if (which != PA_PREFILL_MMA_SYNC && umma_ok) {
+        const int urc = launch_prefill_umma(out, q, key_cache, value_cache, block_tables,
+                                            context_lens, query_start, max_query_len, num_kv_heads,
+                                            scale, num_seqs, num_q_heads, num_q_tokens, head_dim,
+                                            max_blocks_per_seq, num_blocks, dtype,
+                                            static_cast<cudaStream_t>(stream));
+        if (urc != PA_ERR_UNSUPPORTED || which == PA_PREFILL_TCGEN05) return urc;
+    }
     const int64_t tiles = ((int64_t)max_query_len * group + 63) / 64;
     if (tiles > 65535) return PA_ERR_UNSUPPORTED;
     constexpr int STAGES = 4;
@@ -428,6 +443,7 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.num_q_tokens = num_q_tokens;
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.tiles_per_seq = 0;
     CUtensorMap tmk, tmv;
     if (!encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
         !encode_cache_map(&tmv, value_cache, num_blocks, num_kv_heads, head_dim, dtype))

@@ -734,6 +734,7 @@ struct PrefillArgs {
     int max_blocks_per_seq;
     int num_q_tokens;
     float scale_log2;
+    int tiles_per_seq;  // tcgen05 kernel: CTAs per (sequence, kv head)
 };
 
 constexpr float kMaskedLogit = -1.0e30f;  // finite, so 2^(masked - max) is exactly 0

@@ -523,6 +523,21 @@ def test_prefill_bad_block_id_is_reported(prefill_kernel):
     assert gh.max_excess(out[64:], ref, wl.BF16) <= gh.TOL[wl.BF16]
 
 
+@pytest.mark.parametrize("num_seqs", [40, 300])
+def test_prefill_many_sequences_with_equal_lengths(num_seqs, prefill_kernel):
+    """Many sequences, lengths repeating (ties in the longest-first CTA
+    order); 300 sequences is past the size the tcgen05 kernel ranks, which
+    then keeps the plain order."""
+    rng = wl.rng_for(49 + num_seqs)
+    lens = np.array([(17, 200, 64, 1, 130)[i % 5] for i in range(num_seqs)], np.int32)
+    qlens = np.minimum(lens, np.array([(5, 64, 64, 1, 40)[i % 5] for i in range(num_seqs)], np.int32))
+    p = make_paged(rng, num_seqs, 8, 2, 64, lens, wl.blocks_needed(lens, 16) + 1, wl.F16)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), 8, 64), wl.F16)
+    out, ref = run_prefill(p, qchunk, qlens)
+    assert pk.get_error() == (0, 0)
+    assert gh.max_excess(out, ref, wl.F16) <= gh.TOL[wl.F16]
+
+
 def test_prefill_kernels_agree():
     """The two prefill kernels on one problem: both within the budget of
     the oracle, and within twice that budget of each other."""

@@ -41,3 +41,18 @@ def test_descriptor_encodings_match_cutlass(tmp_path):
                            "-o", exe, os.path.join(ROOT, "tests", "umma_encoding_check.cu")])
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
+
+
+def test_fma_pipe_exp2_accuracy(tmp_path):
+    """The polynomial 2^a the tcgen05 softmax runs beside the special-function
+    unit: relative error below 1e-4 on [-125, 8] against double precision,
+    and tiny positive values below -125 (masked scores)."""
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    exe = str(tmp_path / "exp2_fma_check")
+    subprocess.check_call([nvcc, "-std=c++17", "-O2",
+                           "-I", os.path.join(ROOT, "paged_kv_cache_425_b200", "csrc"),
+                           "-o", exe, os.path.join(ROOT, "tests", "exp2_fma_check.cu")])
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.startswith("ok"), r.stdout + r.stderr
