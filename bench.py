@@ -132,12 +132,23 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_digest() -> str:
+DECODE_SOURCE_END = b"// ------------------------------------------------------------------ chunked prefill"
+
+
+def decode_source_digest(read=None) -> str:
+    """Hash of the source the decode, scatter, copy and merge kernels are built
+    from: the device helpers and the kernel header up to its chunked-prefill
+    section.  `read(name) -> bytes` reads a source file (default: this tree)."""
     import hashlib
+    if read is None:
+        def read(name):
+            with open(os.path.join(ROOT, "paged_kv_cache_425_b200", "csrc", name), "rb") as fh:
+                return fh.read()
+    kernels = read("pa_kernels.cuh")
+    cut = kernels.find(DECODE_SOURCE_END)
     h = hashlib.sha256()
-    for f in ("pa_kernels.cuh", "pa_device.cuh"):
-        with open(os.path.join(ROOT, "paged_kv_cache_425_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    h.update(kernels[:cut] if cut >= 0 else kernels)
+    h.update(read("pa_device.cuh"))
     return h.hexdigest()[:16]
 
 
@@ -149,7 +160,7 @@ def traffic_per_call(workload: str, calls_bytes: int):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("source_digest") != kernel_source_digest():
+    if rec.get("source_digest") != decode_source_digest():
         return None
     r = rec.get("workloads", {}).get(workload)
     if not r:
