@@ -61,7 +61,7 @@ constexpr uint32_t kUmmaTmemCols = 512;
 constexpr float kMaxSlack = 8.f;       // log2 growth of the max tolerated before a rescale
 constexpr int kRankMax = 256;          // batches up to this size are scheduled longest first
 #ifndef PA_EXP2_FMA_EVERY
-#define PA_EXP2_FMA_EVERY 0
+#define PA_EXP2_FMA_EVERY 8
 #endif
 // One softmax weight pair in this many is computed on the FMA pipe
 // (exp2_fma_pair) instead of the special-function unit; 0 = none.
@@ -85,6 +85,12 @@ template <>
 struct UmmaFormat<__nv_bfloat16> {
     static constexpr uint32_t value = 1;
 };
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 // Wait for phase `parity` of `bar`; give up when the CTA's abort flag is
 // raised, or after kWaitTimeoutNs (then raise it and flag PA_DEVERR_TIMEOUT).
@@ -181,6 +187,20 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int ntiles = (nkeys + kUmmaKeys - 1) / kUmmaKeys;
     const int32_t *trow = a.block_tables + (size_t)s * a.max_blocks_per_seq;
 
+    // The producer thread sets up the barriers and starts the query-tile load
+    // before the CTA stages its block ids, so its latency overlaps the setup.
+    if (warp == 8 && lane == 0) {
+        for (int i = 0; i < 15; ++i) mbar_init(&bar[i], (i == 11 || i == 12) ? 4 : 1);
+        fence_mbar_init();
+        s_abort = 0;
+        mbar_arrive_expect_tx(q_full, (uint32_t)(kUmmaQTiles * NCH * rows_used * 128));
+#pragma unroll
+        for (int k = 0; k < kUmmaQTiles; ++k)
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+                tma_load_4d(sq + k * QB + c * kUmmaChunk, &tmq, q_full, c * 64, 0, kvh,
+                            q0 + (tile * kUmmaQTiles + k) * TT);
+    }
     // the CTA's block ids, checked once: -1 marks an id out of range
     for (int i = tid; i < nblk; i += kUmmaThreads) {
         int b = trow[i];
@@ -189,11 +209,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             b = -1;
         }
         s_table[i] = b;
-    }
-    if (tid == 0) {
-        for (int i = 0; i < 15; ++i) mbar_init(&bar[i], (i == 11 || i == 12) ? 4 : 1);
-        fence_mbar_init();
-        s_abort = 0;
     }
     if (warp == 8) {
         tmem_alloc(&s_tmem, kUmmaTmemCols);
@@ -208,62 +223,45 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // warpgroup holds until exit, and the teardown is repeated per branch.
     if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-    if (warp == 8) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            bool ok = true;
-            int k_issued = 0, v_issued = 0;
-            mbar_arrive_expect_tx(q_full, (uint32_t)(kUmmaQTiles * NCH * rows_used * 128));
-#pragma unroll
-            for (int k = 0; k < kUmmaQTiles; ++k)
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-                    tma_load_4d(sq + k * QB + c * kUmmaChunk, &tmq, q_full, c * 64, 0, kvh,
-                                q0 + (tile * kUmmaQTiles + k) * TT);
-            for (int j = 0; j < ntiles; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                int nvalid = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int blk = j * 8 + i;
-                    nvalid += blk < nblk && s_table[blk] >= 0;
-                }
-                const uint32_t bytes = (uint32_t)(nvalid * kBlock * D * 2);
-                if (j >= 2 && !(ok = wait_or_abort(&k_empty[st], ph ^ 1, abort_flag))) break;
-                mbar_arrive_expect_tx(&k_full[st], bytes);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int blk = j * 8 + i;
-                    const int id = blk < nblk ? s_table[blk] : -1;
-                    if (id >= 0)
-#pragma unroll
-                        for (int c = 0; c < NCH; ++c)
-                            tma_load_2d(sk + st * KVB + c * kUmmaChunk + i * 2048, &tmk,
-                                        &k_full[st], c * 64, (id * a.num_kv_heads + kvh) * kBlock);
-                }
-                k_issued = j + 1;
-                if (j >= 2 && !(ok = wait_or_abort(&v_empty[st], ph ^ 1, abort_flag))) break;
-                mbar_arrive_expect_tx(&v_full[st], bytes);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int blk = j * 8 + i;
-                    const int id = blk < nblk ? s_table[blk] : -1;
-                    if (id >= 0)
-#pragma unroll
-                        for (int c = 0; c < NCH; ++c)
-                            tma_load_2d(sv + st * KVB + c * kUmmaChunk + i * 2048, &tmv,
-                                        &v_full[st], c * 64, (id * a.num_kv_heads + kvh) * kBlock);
-                }
-                v_issued = j + 1;
+    if (warp == 8 || warp == 10) {
+        // ------------------------------------------------------------ producers
+        // warp 8 fills the K ring, warp 10 the V ring.  A key tile is 8 blocks
+        // x NCH boxes of 16 rows x 128 bytes; lane l issues box l (block l / NCH,
+        // chunk l % NCH), so the TMA unit sees the tile's boxes from parallel
+        // lanes, not one thread's serial stream (one issuing thread leaves it
+        // well short of the rate the GEMMs consume K and V at).
+        const bool is_k = warp == 8;
+        const CUtensorMap *map = is_k ? &tmk : &tmv;
+        uint64_t *full = is_k ? k_full : v_full;
+        uint64_t *empty = is_k ? k_empty : v_empty;
+        uint8_t *ring = is_k ? sk : sv;
+        constexpr int BOXES = 8 * NCH;
+        const int bi = lane / NCH, bc = lane % NCH;
+        bool ok = true;
+        int issued = 0;
+        for (int j = 0; j < ntiles; ++j) {
+            const int st = j & 1;
+            const uint32_t ph = (j >> 1) & 1;
+            const int blk = j * 8 + bi;
+            const int id = (lane < BOXES && blk < nblk) ? s_table[blk] : -1;
+            const uint32_t nbox = __popc(__ballot_sync(FULL, id >= 0));
+            if (j >= 2) {
+                bool freed = true;
+                if (lane == 0) freed = wait_or_abort(&empty[st], ph ^ 1, abort_flag);
+                ok = __shfl_sync(FULL, freed, 0);
+                if (!ok) break;
             }
-            if (!ok) {  // let the copies already issued land before the CTA exits
-                mbar_wait_bounded(q_full, 0, kWaitTimeoutNs);
-                for (int j = max(0, k_issued - 2); j < k_issued; ++j)
-                    mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1, kWaitTimeoutNs);
-                for (int j = max(0, v_issued - 2); j < v_issued; ++j)
-                    mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, kWaitTimeoutNs);
-            }
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], nbox * (uint32_t)(kBlock * 128));
+            __syncwarp();
+            if (id >= 0)
+                tma_load_2d(ring + st * KVB + bc * kUmmaChunk + bi * 2048, map, &full[st], bc * 64,
+                            (id * a.num_kv_heads + kvh) * kBlock);
+            issued = j + 1;
+        }
+        if (!ok && lane == 0) {  // let the copies already issued land before the CTA exits
+            if (is_k) mbar_wait_bounded(q_full, 0, kWaitTimeoutNs);
+            for (int j = max(0, issued - 2); j < issued; ++j)
+                mbar_wait_bounded(&full[j & 1], (j >> 1) & 1, kWaitTimeoutNs);
         }
         __syncwarp();
     } else if (warp == 9) {
@@ -373,21 +371,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                 const int blk = j * 8 + q;
                 if (blk < nblk && s_table[blk] < 0) bad |= 1u << q;
             }
-            // the max of the raw scores (scale > 0 keeps the order)
+            // the max of the raw scores (scale > 0 keeps the order); three-input
+            // max, four independent chains
             float mx4[4] = {kMaskedLogit, kMaskedLogit, kMaskedLogit, kMaskedLogit};
             if (key0 + kUmmaKeys - 1 > pos || bad) {
 #pragma unroll
                 for (int c = 0; c < kUmmaKeys; ++c) {
                     const bool masked = key0 + c > pos || ((bad >> (c >> 4)) & 1u);
-                    const float v = masked ? kMaskedLogit : __uint_as_float(x[c]);
-                    x[c] = __float_as_uint(v);
-                    mx4[c & 3] = fmaxf(mx4[c & 3], v);
+                    if (masked) x[c] = __float_as_uint(kMaskedLogit);
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < kUmmaKeys; ++c)
-                    mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(x[c]));
             }
+#pragma unroll
+            for (int c = 0; c < kUmmaKeys; c += 2)
+                mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
             float alpha = 1.f;
             bool rescale = false;
