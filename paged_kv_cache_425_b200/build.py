@@ -23,8 +23,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("pa_api.cu", "pa_alloc.cc", "pa_sim.cc")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_device.cuh")] + [
-    os.path.join(INCLUDE, f) for f in ("pa_api.h", "pa_alloc.h")]
+# every file the library is built from: a change to any header rebuilds it
+DEPS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)) + sorted(
+    os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

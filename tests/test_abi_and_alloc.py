@@ -443,3 +443,16 @@ def test_prefill_select_accepts_the_three_kernels_only():
         pk.prefill_select(name)
     with pytest.raises(ValueError):
         pk.prefill_select("wgmma")
+
+
+def test_build_rebuilds_on_any_source_or_header_change():
+    """The staleness check covers every file the library is compiled from."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "pa_build", os.path.join(ROOT, "paged_kv_cache_425_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    csrc = os.path.join(ROOT, "paged_kv_cache_425_b200", "csrc")
+    want = {os.path.join(csrc, f) for f in os.listdir(csrc)}
+    want |= {os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))}
+    assert want <= set(b.DEPS)
