@@ -137,8 +137,9 @@ DECODE_SOURCE_END = b"// -------------------------------------------------------
 
 def decode_source_digest(read=None) -> str:
     """Hash of the source the decode, scatter, copy and merge kernels are built
-    from: the device helpers and the kernel header up to its chunked-prefill
-    section.  `read(name) -> bytes` reads a source file (default: this tree)."""
+    from: the device helpers, the kernel header up to its chunked-prefill
+    section, and the host's choice of decode kernel for one query head per kv
+    head.  `read(name) -> bytes` reads a source file (default: this tree)."""
     import hashlib
     if read is None:
         def read(name):
@@ -149,6 +150,10 @@ def decode_source_digest(read=None) -> str:
     h = hashlib.sha256()
     h.update(kernels[:cut] if cut >= 0 else kernels)
     h.update(read("pa_device.cuh"))
+    # which kernel the host picks for one query head per kv head
+    for line in read("pa_api.cu").splitlines():
+        if line.startswith(b"#define PA_MHA_ON_MMA"):
+            h.update(line)
     return h.hexdigest()[:16]
 
 

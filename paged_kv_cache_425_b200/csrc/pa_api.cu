@@ -29,7 +29,7 @@ namespace {
 #define PA_STAGES_64 2   // 2 x 4 KiB per warp at head_dim 64
 #endif
 #ifndef PA_MHA_ON_MMA
-#define PA_MHA_ON_MMA 0  // 1: one query head per kv head also takes the mma.sync kernel
+#define PA_MHA_ON_MMA 1  // 0: one query head per kv head takes the f32 CUDA-core kernel
 #endif
 constexpr int kWarps = PA_DECODE_WARPS;
 constexpr int kStages128 = PA_STAGES_128;
