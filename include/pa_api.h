@@ -127,7 +127,10 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
  *   K_j = key_cache  [block_tables[s][j / 16]][g][j % 16][:],  j < L
  *   V_j = value_cache[block_tables[s][j / 16]][g][j % 16][:]
  *   out[s][h][:] = sum_j softmax_j(scale * q[s][h] . K_j) V_j
- * Products and the softmax are computed in fp32; out is rounded to dtype.
+ * q . K products accumulate in fp32 and the softmax runs in fp32; the P . V
+ * product takes P rounded to dtype (tensor cores; built with PA_MHA_ON_MMA=0,
+ * one query head per kv head keeps P in fp32 on CUDA cores); out is rounded
+ * to dtype.
  * L == 0 gives a zero row.  Table entries past ceil(L / 16) are not read.
  *
  * Contexts longer than PA_PARTITION_TOKENS are split into partitions that

@@ -4,10 +4,12 @@
 //                          vector of a new token's K and V rows.
 //  * copy_blocks_kernel  - pa_copy_blocks: 16-byte vector copy of whole
 //                          blocks (all kv heads, K and V).
-//  * decode_simt_kernel  - pa_decode with one query head per kv head.
-//  * decode_mma_kernel   - pa_decode with 2..16 query heads per kv head: the
+//  * decode_mma_kernel   - pa_decode with 1..16 query heads per kv head: the
 //                          query group is one mma.sync tile against each
-//                          16-token K / V tile.
+//                          16-token K / V tile (the default for every group).
+//  * decode_simt_kernel  - pa_decode with one query head per kv head on f32
+//                          CUDA cores (selected when built with
+//                          PA_MHA_ON_MMA=0).
 //  * merge_kernel        - log-sum-exp merge of the partitions of contexts
 //                          longer than one partition.
 //
