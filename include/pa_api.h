@@ -73,7 +73,8 @@ typedef enum {
 typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 
 #define PA_BLOCK_SIZE 16
-/* Decode splits a context into partitions of this many tokens (32 blocks). */
+/* Decode splits a context into partitions of this many tokens (32 blocks);
+ * calls whose block tables span 16384 tokens or more use twice that. */
 #ifndef PA_PARTITION_TOKENS
 #define PA_PARTITION_TOKENS 512
 #endif
@@ -133,7 +134,8 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
  * to dtype.
  * L == 0 gives a zero row.  Table entries past ceil(L / 16) are not read.
  *
- * Contexts longer than PA_PARTITION_TOKENS are split into partitions that
+ * Contexts longer than one partition (PA_PARTITION_TOKENS tokens, or twice
+ * that when max_blocks_per_seq * 16 >= 16384) are split into partitions that
  * run in parallel and are merged by log-sum-exp; the partial results go to
  * `workspace`, which must hold pa_decode_workspace_size(...) bytes (256-byte
  * aligned) whenever max_blocks_per_seq * 16 > PA_PARTITION_TOKENS, and may be

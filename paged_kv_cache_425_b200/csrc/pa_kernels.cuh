@@ -16,7 +16,8 @@
 // Decode grid: x = sequence * Hkv + kv head, y = partition (slowest, so the
 // CTAs of partitions past a short sequence's end, which exit at once, come
 // last and overlap the tail of the grid).  A partition covers
-// PA_PARTITION_TOKENS tokens (32 blocks).  Inside a CTA each warp owns every
+// PA_PARTITION_TOKENS tokens (32 blocks), or twice that for calls whose block
+// tables span 16384 tokens or more (a.part_blocks).  Inside a CTA each warp owns every
 // NW-th block of the partition and runs its own STAGES-deep TMA pipeline:
 // one lane loads the warp's next (block, kv head) K and V tiles with
 // cp.async.bulk.tensor into a 128-byte-swizzled shared-memory stage and an
@@ -57,6 +58,8 @@ struct DecodeArgs {
     int num_kv_heads;
     int max_blocks_per_seq;
     int num_parts;     // partitions per sequence in the grid
+    int part_blocks;   // blocks per partition for this call (the decode kernels
+                       // also take it as their PB template argument)
     float scale_log2;  // scale * log2(e)
 };
 
@@ -176,7 +179,7 @@ __device__ __forceinline__ int warp_block_count(int nb_local, int warp, int nw) 
 }
 
 // ------------------------------------------------------------------ decode: one q head per kv head
-template <typename T, int D, int NW, int STAGES>
+template <typename T, int D, int NW, int STAGES, int PB>
 __global__ void __launch_bounds__(NW * 32)
     decode_simt_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const DecodeArgs a) {
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(NW * 32)
     pdl_wait_prior();
     const int L = clamp_context(a, s, part == 0 && kvh == 0 && threadIdx.x == 0);
     const int nblk = (L + kBlock - 1) / kBlock;
-    const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
+    const int nparts = (nblk + PB - 1) / PB;
     if (part >= (nparts > 0 ? nparts : 1)) return;
     const size_t row = (size_t)s * a.num_q_heads + kvh;  // q head == kv head
     uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + row * D;
@@ -204,8 +207,8 @@ __global__ void __launch_bounds__(NW * 32)
         for (int i = threadIdx.x; i < D; i += NW * 32) out[i] = 0;
         return;
     }
-    const int b_begin = part * kPartBlocks;
-    const int nb_local = min(kPartBlocks, nblk - b_begin);
+    const int b_begin = part * PB;
+    const int nb_local = min(PB, nblk - b_begin);
     const int nk = warp_block_count(nb_local, warp, NW);
 
     Pipe pipe;
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(NW * 32)
 
 // ------------------------------------------------------------------ decode: query group on mma.sync
 // NT = number of 8-head column tiles (G <= 8 * NT).
-template <typename T, int D, int NW, int STAGES, int NT>
+template <typename T, int D, int NW, int STAGES, int NT, int PB>
 __global__ void __launch_bounds__(NW * 32)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a) {
@@ -388,7 +391,7 @@ __global__ void __launch_bounds__(NW * 32)
     pdl_wait_prior();
     const int L = clamp_context(a, s, part == 0 && kvh == 0 && threadIdx.x == 0);
     const int nblk = (L + kBlock - 1) / kBlock;
-    const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
+    const int nparts = (nblk + PB - 1) / PB;
     if (part >= (nparts > 0 ? nparts : 1)) return;
     const size_t row0 = (size_t)s * a.num_q_heads + (size_t)kvh * G;  // first q head of the group
     uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + row0 * D;
@@ -396,8 +399,8 @@ __global__ void __launch_bounds__(NW * 32)
         for (int i = threadIdx.x; i < G * D; i += NW * 32) out[i] = 0;
         return;
     }
-    const int b_begin = part * kPartBlocks;
-    const int nb_local = min(kPartBlocks, nblk - b_begin);
+    const int b_begin = part * PB;
+    const int nb_local = min(PB, nblk - b_begin);
     const int nk = warp_block_count(nb_local, warp, NW);
 
     Pipe pipe;
@@ -612,7 +615,7 @@ __global__ void __launch_bounds__(kMergeRows * 32) merge_kernel(const DecodeArgs
     const int s = (int)(row / a.num_q_heads);
     const int L = clamp_context(a, s, false);
     const int nblk = (L + kBlock - 1) / kBlock;
-    const int nparts = (nblk + kPartBlocks - 1) / kPartBlocks;
+    const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
     if (nparts <= 1) return;
     const float2 *ml = a.ws_ml + row * a.num_parts;
     float M = -INFINITY;

@@ -82,8 +82,22 @@ def test_every_context_length_1_to_64(hq, hkv, d, dtype):
     assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[dtype]
 
 
+@pytest.mark.parametrize("hq,hkv,dtype", [(8, 8, wl.F16), (16, 4, wl.BF16)])
+def test_tables_at_the_wide_partition_threshold(hq, hkv, dtype):
+    """Tables of 1023 blocks keep 512-token partitions; 1024 blocks (16384
+    tokens) switch to 1024-token ones.  Contexts straddle both boundary sets."""
+    lens = np.array([1, 511, 512, 513, 1023, 1024, 1025, 2047, 2049, 15000], np.int32)
+    for width in (1023, 1024):
+        rng = wl.rng_for(12 + width)
+        L = np.minimum(lens, width * 16)
+        p = make_paged(rng, len(L), hq, hkv, 128, L, wl.blocks_needed(L, 16) + 2, dtype,
+                       max_blocks=width)
+        assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[dtype], width
+
+
 def test_wide_table_many_partitions():
-    """Table width 2048 blocks (64 partitions) with short and long contexts."""
+    """Table width 2048 blocks (32 partitions of 1024 tokens) with short and
+    long contexts."""
     rng = wl.rng_for(8)
     lens = np.array([5, 8192, 32768, 513, 20000], np.int32)
     nb = wl.blocks_needed(lens, 16) + 3
