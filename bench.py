@@ -429,12 +429,13 @@ def run_ours(args, world, rank, local):
 
 def run_e2e(st, args, device, world, chunks: int = 4):
     """Same steps, with every step's inputs copied from pinned host memory and
-    its outputs read back, inside the timed region.  A copy stream moves the
-    inputs of the next group of layers while the current group computes, and
-    reads each group's outputs back as soon as they are done; per-group events
-    keep a step's copies from overwriting buffers the previous step still
-    uses, so one step's last read-back overlaps the next step's compute.  The
-    region ends once the last step's outputs are on the host."""
+    its outputs read back, inside the timed region.  Upload and read-back
+    streams move the inputs of the next group of layers while the current
+    group computes and read each group's outputs back as soon as they are
+    done; per-group events keep a step's copies from overwriting buffers the
+    previous step still uses, so copies of one step overlap the compute of
+    its neighbours.  The region ends once the last step's outputs are on the
+    host."""
     import torch
     L = st.layers
     per = (L + chunks - 1) // chunks
@@ -450,7 +451,9 @@ def run_e2e(st, args, device, world, chunks: int = 4):
     h2d = sum(h.numel() * h.element_size() for h in (hq, hk, hv)) + \
         sum(h.numel() * h.element_size() for _, h in meta)
     d2h = hout.numel() * hout.element_size()
-    copy = torch.cuda.Stream(device)
+    up = torch.cuda.Stream(device)      # inputs of each layer group, host -> device
+    meta_s = torch.cuda.Stream(device)  # the step's tables, lengths and slots
+    down = torch.cuda.Stream(device)    # each group's outputs, device -> host
     comp = st.stream
     ev_in = [torch.cuda.Event() for _ in groups]      # inputs of a group are on the device
     ev_done = [torch.cuda.Event() for _ in groups]    # a group's compute finished
@@ -470,32 +473,37 @@ def run_e2e(st, args, device, world, chunks: int = 4):
             hout.copy_(st.out, non_blocking=True)
 
     def one_overlapped():
-        with torch.cuda.stream(copy):
+        # Uploads, metadata and read-backs each have their own stream, so a
+        # group's upload waits only for the previous step's use of the same
+        # group, and nothing but the small metadata copy sits between the
+        # previous step's last layer and this step's first.
+        with torch.cuda.stream(meta_s):
             if not first[0]:
-                copy.wait_event(ev_meta_free)
+                meta_s.wait_event(ev_meta_free)   # previous step no longer reads them
             for dev, host in meta:
                 dev.copy_(host, non_blocking=True)
-            ev_meta.record(copy)
+            ev_meta.record(meta_s)
+        with torch.cuda.stream(up):
             for c, (a, b) in enumerate(groups):
                 if not first[0]:
-                    copy.wait_event(ev_done[c])       # previous step no longer reads them
+                    up.wait_event(ev_done[c])     # previous step no longer reads them
                 st.q[a:b].copy_(hq[a:b], non_blocking=True)
                 st.k_new[a:b].copy_(hk[a:b], non_blocking=True)
                 st.v_new[a:b].copy_(hv[a:b], non_blocking=True)
-                ev_in[c].record(copy)
+                ev_in[c].record(up)
         comp.wait_event(ev_meta)
         for c, (a, b) in enumerate(groups):
             comp.wait_event(ev_in[c])
             if not first[0]:
-                comp.wait_event(ev_read[c])           # previous outputs are read back
+                comp.wait_event(ev_read[c])       # previous outputs are read back
             st.step_layers(a, b)
             ev_done[c].record(comp)
         ev_meta_free.record(comp)
-        with torch.cuda.stream(copy):
+        with torch.cuda.stream(down):
             for c, (a, b) in enumerate(groups):
-                copy.wait_event(ev_done[c])
+                down.wait_event(ev_done[c])
                 hout[a:b].copy_(st.out[a:b], non_blocking=True)
-                ev_read[c].record(copy)
+                ev_read[c].record(down)
         first[0] = False
 
     # with one layer group there is nothing to overlap: one stream, no syncs
@@ -526,7 +534,7 @@ def run_e2e(st, args, device, world, chunks: int = 4):
     return {"value": round(world * st.S * args.steps / (ms * 1e-3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms / args.steps, 4),
-            "overlap": (f"copy stream, {len(groups)} layer groups" if len(groups) > 1
+            "overlap": (f"upload, metadata and read-back streams, {len(groups)} layer groups" if len(groups) > 1
                         else "none (one layer): copies and kernels on one stream")}
 
 
