@@ -53,6 +53,17 @@ def test_workspace_size_rule():
     assert pk.decode_workspace_size(64, 32, 128, 128, block_size=32) == 0
 
 
+def test_workspace_follows_the_partition_rule():
+    """Tables spanning 16384 tokens or more use 1024-token partitions: half as
+    many partials per row as 512-token ones."""
+    def rows_parts(max_blocks):
+        n = pk.decode_workspace_size(8, 8, 128, max_blocks)
+        return n // (8 * 8 * (128 * 4 + 8))  # lower bound on partitions per row
+    assert rows_parts(1023) == 32          # 16368 tokens: 512-token partitions
+    assert rows_parts(1024) == 16          # 16384 tokens: 1024-token partitions
+    assert rows_parts(2048) == 32
+
+
 def test_import_fails_loudly_without_the_library(tmp_path):
     dst = tmp_path / "paged_kv_cache_425_b200"
     shutil.copytree(os.path.join(ROOT, "paged_kv_cache_425_b200"), dst,
