@@ -154,6 +154,28 @@ bool set_smem(Kernel k, int bytes) {
     return true;
 }
 
+// Registers per thread a kernel was compiled with (-1 on failure); looked up
+// once per kernel and device.
+template <typename Kernel>
+int compiled_registers(Kernel k) {
+    struct Entry {
+        const void *fn;
+        int dev, regs;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> seen;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    const void *fn = reinterpret_cast<const void *>(k);
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &e : seen)
+        if (e.fn == fn && e.dev == dev) return e.regs;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return -1;
+    seen.push_back({fn, dev, fa.numRegs});
+    return fa.numRegs;
+}
+
 template <typename T, int D, int PB>
 int launch_decode(const DecodeArgs &a, int group, const CUtensorMap &tmk, const CUtensorMap &tmv,
                   cudaStream_t st) {
@@ -289,9 +311,9 @@ int launch_prefill_umma(void *out, const void *q, const void *key_cache, const v
         // the kernel re-splits its registers per warpgroup (setmaxnreg); a
         // split above what the launch holds would wait forever, so check the
         // compiled count first
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return PA_ERR_CUDA;
-        if ((int64_t)fa.numRegs * kUmmaThreads < kUmmaRegsNeeded) return PA_ERR_UNSUPPORTED;
+        const int regs = compiled_registers(kernel);
+        if (regs < 0) return PA_ERR_CUDA;
+        if ((int64_t)regs * kUmmaThreads < kUmmaRegsNeeded) return PA_ERR_UNSUPPORTED;
         if (!set_smem(kernel, smem)) return PA_ERR_CUDA;
         return launch_pdl(kernel, grid, dim3(kUmmaThreads), (size_t)smem, st, tmq, tmk, tmv, a);
     };
