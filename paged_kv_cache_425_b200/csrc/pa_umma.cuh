@@ -152,23 +152,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 #undef PA_TMEM_R8
 
-// Warp-wide store of 32 lanes x 64 columns; the caller waits with
+// Warp-wide stores of 32 lanes x N columns; the caller waits with
 // tmem_wait_st() before signalling the stored values to another thread.
 #define PA_TMEM_W8(b) "r"(r[b + 0]), "r"(r[b + 1]), "r"(r[b + 2]), "r"(r[b + 3]), \
                       "r"(r[b + 4]), "r"(r[b + 5]), "r"(r[b + 6]), "r"(r[b + 7])
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
-        "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
-        "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
-        PA_TMEM_W8(0), PA_TMEM_W8(8), PA_TMEM_W8(16), PA_TMEM_W8(24), PA_TMEM_W8(32),
-        PA_TMEM_W8(40), PA_TMEM_W8(48), PA_TMEM_W8(56)
-        : "memory");
-}
-
-// The same for 32 columns.
+// 32 columns.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
