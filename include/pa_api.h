@@ -232,12 +232,16 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *
  * Limits and rules:
- *  - If pa_decode_workspace_size(...) for these sizes exceeds
- *    PA_STATIC_WORKSPACE_BYTES, the call returns PA_ERR_WORKSPACE and
- *    enqueues nothing.
+ *  - The arguments are checked first, exactly as pa_decode checks them, so
+ *    the two calls return the same status for the same arguments.  Then, if
+ *    pa_decode_workspace_size(...) for these sizes exceeds
+ *    PA_STATIC_WORKSPACE_BYTES, the call returns PA_ERR_WORKSPACE.  A call
+ *    that returns an error enqueues nothing.
  *  - The first call on a device looks up the array's device address (once
- *    per device, with that device current).  Make that first call before any
- *    stream capture begins.
+ *    per device and CUDA context, with that device current).  Make that first
+ *    call before any stream capture begins.  After a cudaDeviceReset the old
+ *    address belongs to a context that no longer exists; the next call, in the
+ *    new context, looks the address up again (so it is again a first call).
  *  - All calls share the one array, and it keeps the last call's contents.
  *    Nothing in it has to start at zero.  Calls that overlap on the GPU
  *    (other streams, other host threads) race on the array and give wrong

@@ -364,26 +364,56 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
     return (size_t)workspace_layout(num_seqs, num_q_heads, head_dim, parts).total;
 }
 
-int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
-              const int32_t *block_tables, const int32_t *context_lens, int32_t num_kv_heads,
-              float scale, int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
-              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
-              void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace pa {
+namespace {
+// Host-side checks of a decode call's arguments, in the order pa_decode
+// applies them (shared with pa_decode_static_workspace, so both return the
+// same status for the same arguments).  PA_OK with *empty set means there is
+// nothing to launch.
+int check_decode_args(const void *out, const void *q, const void *key_cache,
+                      const void *value_cache, const int32_t *block_tables,
+                      const int32_t *context_lens, int32_t num_kv_heads, int32_t num_seqs,
+                      int32_t num_q_heads, int32_t head_dim, int32_t block_size,
+                      int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype, bool *empty) {
+    *empty = false;
     int rc = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int group = num_q_heads / num_kv_heads;
     if (group > 16) return PA_ERR_UNSUPPORTED;
-    if (num_seqs == 0) return PA_OK;
+    if (num_seqs == 0) {
+        *empty = true;
+        return PA_OK;
+    }
     if ((int64_t)num_seqs * num_q_heads >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
         return PA_ERR_INVALID_ARG;
     if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || !aligned(q, 8) ||
         !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
         return PA_ERR_INVALID_ARG;
+    if (num_parts_for(max_blocks_per_seq) > 8192) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *context_lens, int32_t num_kv_heads,
+              float scale, int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
+              void *workspace, size_t workspace_bytes, void *stream) {
+    bool empty = false;
+    const int rc = check_decode_args(out, q, key_cache, value_cache, block_tables, context_lens,
+                                     num_kv_heads, num_seqs, num_q_heads, head_dim, block_size,
+                                     max_blocks_per_seq, num_blocks, dtype, &empty);
+    if (rc != PA_OK || empty) return rc;
+    const int group = num_q_heads / num_kv_heads;
     const int64_t parts = num_parts_for(max_blocks_per_seq);
-    if (parts > 8192) return PA_ERR_UNSUPPORTED;
 
     DecodeArgs a;
     a.out = out;
@@ -628,27 +658,65 @@ int pa_version(void) { return 100; }
 // Scratch of pa_decode_static_workspace, for callers that cannot allocate
 // device memory (see include/pa_api.h).  In host code `g_static_workspace`
 // names a host-side stand-in, not a device address: its device address is
-// looked up with cudaGetSymbolAddress, once per device, with that device
-// current.
+// looked up with cudaGetSymbolAddress, once per device and CUDA context, with
+// that device current.
 namespace {
 
 static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mutex;
-void *g_static_address[kMaxDevices] = {};
+struct StaticAddress {
+    void *ptr;
+    unsigned long long ctx_id;  // the context the address belongs to
+};
+StaticAddress g_static_address[kMaxDevices] = {};
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (ids are never reused
+// within a process, unlike context handles), or 0 when there is none yet or
+// the driver cannot say.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the array in the current device's current context.  A
+// device reset (cudaDeviceReset) ends the context the cached address belongs
+// to; the next call, in the new context, looks the address up again.
 int static_workspace_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_static_mutex);
-    if (!g_static_address[dev]) {
+    StaticAddress &e = g_static_address[dev];
+    const unsigned long long id = current_context_id();
+    if (!e.ptr || id == 0 || id != e.ctx_id) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return PA_ERR_CUDA;
-        g_static_address[dev] = p;
+        e.ptr = p;
+        e.ctx_id = current_context_id();  // the lookup makes the primary context current
     }
-    *out = g_static_address[dev];
+    *out = e.ptr;
     return PA_OK;
 }
 
@@ -661,6 +729,13 @@ extern "C" int pa_decode_static_workspace(void *out, const void *q, const void *
                                           int32_t head_dim, int32_t block_size,
                                           int32_t max_blocks_per_seq, int64_t num_blocks,
                                           int32_t dtype, void *stream) {
+    // the same argument checks as pa_decode, first, so both give the same
+    // status for the same arguments; then the array's size
+    bool empty = false;
+    const int vrc = check_decode_args(out, q, key_cache, value_cache, block_tables, context_lens,
+                                      num_kv_heads, num_seqs, num_q_heads, head_dim, block_size,
+                                      max_blocks_per_seq, num_blocks, dtype, &empty);
+    if (vrc != PA_OK || empty) return vrc;
     const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, block_size,
                                                  max_blocks_per_seq);
     if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;

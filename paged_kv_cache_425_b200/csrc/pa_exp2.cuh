@@ -11,11 +11,14 @@
 //         2^f on 2000 Chebyshev nodes of [-0.5, 0.5] with relative weights:
 //         relative error below 8e-5 in float32 Horner evaluation, under the
 //         rounding of the 16-bit P it feeds (2^-9 bf16, 2^-11 f16);
-//   2^a = 2^f with n added to its exponent field.
-// Inputs are clamped at -125 so the exponent field stays normal; 2^-125 (and
-// anything below, masked scores included) then comes out as about 2^-125
-// rather than 0.  A softmax row's weight sum is at least 1 (its max scores
-// 2^0), so such a weight is over 120 binary orders below it.
+//   2^a = 2^f * 2^n, with 2^n built directly in the exponent field of 1.0;
+//         the product is exact (2^f is in [0.7, 1.42] and n >= -125, so it
+//         stays a normal number), and a NaN input stays NaN through it.
+// Inputs are clamped at -125 so 2^n stays normal; 2^-125 (and anything
+// below, masked scores included) then comes out as about 2^-125 rather than
+// 0.  A softmax row's weight sum is at least 1 (its max scores 2^0), so such
+// a weight is over 120 binary orders below it.  The clamp is a comparison
+// that is false for NaN, so NaN is not clamped away.
 #pragma once
 
 #include <cstdint>
@@ -49,12 +52,14 @@ PA_HD inline float f32_from(uint32_t u) {
 
 // Scalar form: the same operations, in the same order, as exp2_fma_pair.
 PA_HD inline float exp2_fma(float a) {
-    a = a > kExp2Min ? a : kExp2Min;
+    a = a < kExp2Min ? kExp2Min : a;  // NaN passes (the comparison is false)
     const float nf = a + kExp2Round;
     const float n = nf - kExp2Round;
     const float f = fmaf(n, -1.f, a);
     const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-    return f32_from(f32_bits(p) + (f32_bits(nf) << 23));
+    // the low mantissa bits of nf hold n: shifted into the exponent field of
+    // 1.0 they give 2^n
+    return p * f32_from((f32_bits(nf) << 23) + 0x3f800000u);
 }
 
 #if defined(__CUDACC__)
@@ -76,21 +81,26 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 
 // exp2_fma on two values with paired (f32x2) arithmetic.
 __device__ __forceinline__ void exp2_fma_pair(float a0, float a1, float &p0, float &p1) {
-    const uint64_t a = f32x2_pack(fmaxf(a0, kExp2Min), fmaxf(a1, kExp2Min));
+    const uint64_t a = f32x2_pack(a0 < kExp2Min ? kExp2Min : a0, a1 < kExp2Min ? kExp2Min : a1);
     const uint64_t nf = f32x2_add(a, f32x2_pack(kExp2Round, kExp2Round));
     const uint64_t n = f32x2_add(nf, f32x2_pack(-kExp2Round, -kExp2Round));
     const uint64_t f = f32x2_fma(n, f32x2_pack(-1.f, -1.f), a);
     uint64_t p = f32x2_fma(f32x2_pack(kExp2C3, kExp2C3), f, f32x2_pack(kExp2C2, kExp2C2));
     p = f32x2_fma(p, f, f32x2_pack(kExp2C1, kExp2C1));
     p = f32x2_fma(p, f, f32x2_pack(kExp2C0, kExp2C0));
-    float q0, q1, m0, m1;
-    f32x2_unpack(p, q0, q1);
+    float m0, m1;
     f32x2_unpack(nf, m0, m1);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(m0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(m1) << 23));
+    const uint64_t two_n = f32x2_pack(__uint_as_float((__float_as_uint(m0) << 23) + 0x3f800000u),
+                                      __uint_as_float((__float_as_uint(m1) << 23) + 0x3f800000u));
+    f32x2_unpack(f32x2_mul(p, two_n), p0, p1);
 }
 #endif
 

@@ -467,3 +467,29 @@ def test_build_rebuilds_on_any_source_or_header_change():
     want = {os.path.join(csrc, f) for f in os.listdir(csrc)}
     want |= {os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))}
     assert want <= set(b.DEPS)
+
+
+def test_static_workspace_decode_checks_arguments_like_pa_decode():
+    """pa_decode_static_workspace applies pa_decode's argument checks before
+    its own size limit, so both return the same status for the same bad
+    arguments, even at sizes far beyond the static array (host checks only:
+    nothing reaches a device)."""
+    huge_s, d, maxb, nb = 1 << 20, 128, 4096, 1024
+    cases = [
+        (64, 2),            # a query group of 32 heads: unsupported
+        (30, 4),            # 30 q heads over 4 kv heads: invalid
+    ]
+    for hq, hkv in cases:
+        a = pk.pa_decode(None, None, None, None, None, None, hkv, 0.1, huge_s, hq, d, 16, maxb,
+                         nb, pk.F16, None, 0, None)
+        b = pk.pa_decode_static_workspace(None, None, None, None, None, None, hkv, 0.1, huge_s,
+                                          hq, d, 16, maxb, nb, pk.F16, None)
+        assert a == b and a in (pk.PA_ERR_UNSUPPORTED, pk.PA_ERR_INVALID_ARG), (hq, hkv, a, b)
+    # more than 8192 partitions per sequence: unsupported on both.  The
+    # pointers are aligned placeholders: the call returns before any launch
+    # and never dereferences them.
+    wide = 8193 * 64
+    fake = [4096 * (i + 1) for i in range(6)]
+    a = pk.pa_decode(*fake, 8, 0.1, 4, 32, d, 16, wide, nb, pk.BF16, None, 0, None)
+    b = pk.pa_decode_static_workspace(*fake, 8, 0.1, 4, 32, d, 16, wide, nb, pk.BF16, None)
+    assert a == b == pk.PA_ERR_UNSUPPORTED

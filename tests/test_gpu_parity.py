@@ -376,7 +376,14 @@ def test_swap_out_and_back_in_is_bit_exact_and_decode_follows(pinned):
     pk.swap_blocks(dkc, dvc, host_k, host_v, out_pairs)
     torch.cuda.synchronize()
     hk = host_k.view(torch.int16).numpy().view(np.uint16)
-    assert np.array_equal(hk[5:5 + n0], p.key_cache[p.tables[0, :n0]])
+    hv = host_v.view(torch.int16).numpy().view(np.uint16)
+    # the whole host pool: the swapped blocks at their destinations, zeros elsewhere
+    want_hk = np.zeros_like(hk)
+    want_hv = np.zeros_like(hv)
+    for src, dst in out_pairs:
+        want_hk[dst] = p.key_cache[src]
+        want_hv[dst] = p.value_cache[src]
+    assert np.array_equal(hk, want_hk) and np.array_equal(hv, want_hv)
     # back into device blocks no table uses (sequence 1 keeps its blocks)
     used = set(p.tables[:, :].ravel().tolist())
     free = np.array([b for b in range(nb) if b not in used][:n0] if nb - len(used) >= n0 else [], np.int32)
@@ -385,6 +392,14 @@ def test_swap_out_and_back_in_is_bit_exact_and_decode_follows(pinned):
     in_pairs = np.stack([5 + np.arange(n0), free], axis=1).astype(np.int32)
     pk.swap_blocks(host_k, host_v, dkc, dvc, in_pairs)
     torch.cuda.synchronize()
+    # the whole device pool: the destination blocks hold exactly the host
+    # bytes, every other block keeps its own
+    want_k, want_v = p.key_cache.copy(), p.value_cache.copy()
+    for src, dst in in_pairs:
+        want_k[dst] = want_hk[src]
+        want_v[dst] = want_hv[src]
+    assert np.array_equal(gh.to_host_bits(dkc), want_k)
+    assert np.array_equal(gh.to_host_bits(dvc), want_v)
     tables = p.tables.copy()
     tables[0, :n0] = free
     after = gh.to_host_bits(gh.run_decode(pk, p.q, dkc, dvc, tables, lens, H, p.scale, dt))

@@ -4,9 +4,11 @@ Some callers cannot hand pa_decode a workspace: a serving process whose
 device memory is reserved up front by its own pools, a hot loop that must
 not call cudaMalloc (it can synchronise the device), or a foreign-language
 caller with no device allocator.  This entry point uses a fixed array in the
-library instead.  Its output must equal pa_decode's on the same inputs, on
-two calls in a row (the array keeps the first call's contents), and it must
-refuse sizes beyond its array without launching anything.
+library instead.  It launches the same kernels with the same partitioning on
+the same inputs as pa_decode, so its output must be bit-identical to
+pa_decode's, on two calls in a row (the array keeps the first call's
+contents), and within the attention tolerance of the fp64 oracle.  Sizes
+beyond its array must be refused without anything being launched.
 
 The file is named to be collected last, so a run that stops at the first
 failure has already run every other test; it also passes on its own.
@@ -14,6 +16,7 @@ failure has already run every other test; it also passes on its own.
 import numpy as np
 import pytest
 
+import oracle
 import workloads as wl
 from paged_inputs import make_paged
 
@@ -48,8 +51,10 @@ def test_matches_pa_decode_on_two_calls_in_a_row(hq, hkv, dtype):
         p = make_paged(rng, len(lens), hq, hkv, 128, lens, wl.blocks_needed(lens, 16) + 3, dtype)
         assert pk.decode_workspace_size(len(lens), hq, 128, p.tables.shape[1]) > 0
         ref, out = both_ways(p)
-        diff = float((ref.float() - out.float()).abs().max())
-        assert diff <= gh.TOL[dtype], (call, diff)
+        assert torch.equal(ref, out), (call, float((ref.float() - out.float()).abs().max()))
+        want = oracle.decode(p.q, p.key_cache, p.value_cache, p.tables, p.lens, p.num_kv_heads,
+                             p.scale, p.dtype)
+        assert gh.max_err(out, want) <= gh.TOL[dtype], call
     assert pk.get_error() == (0, 0)
 
 
@@ -62,6 +67,12 @@ def test_refuses_sizes_beyond_its_array():
     kc = torch.zeros((4, Hkv, 16, d), dtype=torch.bfloat16, device="cuda")
     tables = torch.zeros((S, maxb), dtype=torch.int32, device="cuda")
     lens = torch.ones(S, dtype=torch.int32, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    torch.cuda.synchronize()
     with pytest.raises(pk.PagedError) as e:
-        pk.decode_static_workspace(q.clone(), q, kc, kc, tables, lens, Hkv, 0.1)
+        pk.decode_static_workspace(out, q, kc, kc, tables, lens, Hkv, 0.1)
     assert e.value.status == pk.PA_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    # nothing ran: the output is untouched and no kernel reported anything
+    assert bool(torch.isnan(out).all())
+    assert pk.get_error() == (0, 0)
