@@ -482,8 +482,9 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
     const int64_t umma_smem = (head_dim == 128 ? prefill_umma_smem_bytes<128>(0)
                                                : prefill_umma_smem_bytes<64>(0)) +
                               4 * (int64_t)max_blocks_per_seq;
+    // (227 KiB per CTA covers static shared memory too: leave 2 KiB for it)
     const bool umma_ok = group <= kUmmaRows && aligned(q, 16) && aligned(out, 16) &&
-                         scale > 0.f && scale < 3.0e38f && umma_smem <= 227 * 1024;
+                         scale > 0.f && scale < 3.0e38f && umma_smem + 2048 <= 227 * 1024;
     if (which == PA_PREFILL_TCGEN05 && !umma_ok) return PA_ERR_UNSUPPORTED;
     if (which != PA_PREFILL_MMA_SYNC && umma_ok) {
         const int urc = launch_prefill_umma(out, q, key_cache, value_cache, block_tables,

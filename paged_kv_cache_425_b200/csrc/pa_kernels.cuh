@@ -39,6 +39,10 @@
 
 #include "pa_device.cuh"
 
+#ifndef PA_DECODE_MIN_CTAS
+#define PA_DECODE_MIN_CTAS 6  // resident CTAs per SM the <= 8-head decode kernel is compiled for
+#endif
+
 namespace pa {
 
 constexpr int kBlock = 16;                                  // tokens per block
@@ -370,9 +374,12 @@ __global__ void __launch_bounds__(NW * 32)
 }
 
 // ------------------------------------------------------------------ decode: query group on mma.sync
-// NT = number of 8-head column tiles (G <= 8 * NT).
+// NT = number of 8-head column tiles (G <= 8 * NT).  With NT == 1 the kernel
+// is compiled for PA_DECODE_MIN_CTAS resident CTAs per SM (80 registers at
+// 6): resident warps, not pipeline depth, set the bandwidth this kernel
+// reaches.
 template <typename T, int D, int NW, int STAGES, int NT, int PB>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, NT == 1 ? PA_DECODE_MIN_CTAS : 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a) {
     using Pipe = WarpPipe<D, STAGES>;

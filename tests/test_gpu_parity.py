@@ -95,6 +95,22 @@ def test_tables_at_the_wide_partition_threshold(hq, hkv, dtype):
         assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[dtype], width
 
 
+@pytest.mark.parametrize("hq,hkv,dtype", [(4, 4, wl.F16), (8, 2, wl.BF16), (16, 1, wl.BF16)])
+def test_two_eight_and_nine_partitions(hq, hkv, dtype):
+    """Tables of 33, 256 and 257 blocks split a context into up to 2, 8 and 9
+    partitions of 512 tokens.  Contexts cover one partition, the partition
+    boundaries, and the whole table."""
+    for width in (33, 256, 257):
+        rng = wl.rng_for(40 + width)
+        cap = width * 16
+        lens = np.array([1, 16, 511, 512, 513, 1024, 1025, 4095, 4096, cap - 1, cap], np.int32)
+        lens = np.minimum(lens, cap)
+        p = make_paged(rng, len(lens), hq, hkv, 128, lens, wl.blocks_needed(lens, 16) + 2, dtype,
+                       max_blocks=width)
+        assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[dtype], width
+    assert pk.get_error() == (0, 0)
+
+
 def test_wide_table_many_partitions():
     """Table width 2048 blocks (32 partitions of 1024 tokens) with short and
     long contexts."""
