@@ -609,8 +609,10 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? PA_DECODE_MIN_CTAS : 1)
 // w_p = l_p 2^(m_p - M), M = max over partitions that saw a token.  Lane i
 // owns partitions i, i + 32, ... for the weights and elements 4i .. 4i + 3 of
 // the row (D / 4 lanes) for the sum; weights travel by shuffle, the partial
-// rows stream in as independent 16-byte loads.  No block barrier.
+// rows stream in as independent 16-byte loads.  No block barrier.  A row of
+// at most kMergeFew partitions issues all its loads before the reduction.
 constexpr int kMergeRows = 4;
+constexpr int kMergeFew = 8;  // rows of at most this many partitions load everything at once
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeRows * 32) merge_kernel(const DecodeArgs a) {
@@ -625,6 +627,39 @@ __global__ void __launch_bounds__(kMergeRows * 32) merge_kernel(const DecodeArgs
     const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
     if (nparts <= 1) return;
     const float2 *ml = a.ws_ml + row * a.num_parts;
+    constexpr int D4 = D / 4;  // float4 pieces of a row
+    const float4 *op = reinterpret_cast<const float4 *>(a.ws_o + row * a.num_parts * D);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+    if (nparts <= kMergeFew) {
+        // every load of the row issued at once (the partial rows do not
+        // depend on the weights): one round trip to L2 instead of two
+        float2 v = lane < nparts ? ml[lane] : make_float2(-INFINITY, 0.f);
+        float4 x[kMergeFew];
+#pragma unroll
+        for (int j = 0; j < kMergeFew; ++j)
+            if (j < nparts && lane < D4) x[j] = op[(size_t)j * D4 + lane];
+        float M = v.y > 0.f ? v.x : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = v.y > 0.f ? v.y * fast_exp2(v.x - M) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kMergeFew; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            den += wj;
+            if (j < nparts && lane < D4) {
+                acc.x += wj * x[j].x; acc.y += wj * x[j].y; acc.z += wj * x[j].z; acc.w += wj * x[j].w;
+            }
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        if (lane < D4) {
+            uint16_t *out = reinterpret_cast<uint16_t *>(a.out) + row * D + 4 * lane;
+            const uint32_t lo = (uint32_t)narrow1(acc.x * inv, T()) | ((uint32_t)narrow1(acc.y * inv, T()) << 16);
+            const uint32_t hi = (uint32_t)narrow1(acc.z * inv, T()) | ((uint32_t)narrow1(acc.w * inv, T()) << 16);
+            *reinterpret_cast<uint2 *>(out) = make_uint2(lo, hi);
+        }
+        return;
+    }
     float M = -INFINITY;
     for (int p = lane; p < nparts; p += 32) {
         const float2 v = ml[p];
@@ -632,10 +667,6 @@ __global__ void __launch_bounds__(kMergeRows * 32) merge_kernel(const DecodeArgs
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    constexpr int D4 = D / 4;  // float4 pieces of a row
-    const float4 *op = reinterpret_cast<const float4 *>(a.ws_o + row * a.num_parts * D);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float den = 0.f;
     for (int p0 = 0; p0 < nparts; p0 += 32) {
         const int p = p0 + lane;
         float w = 0.f;
