@@ -332,15 +332,18 @@ class Setup:
     def step(self):
         self.step_layers(0, self.layers)
 
-    def step_layers(self, first: int, last: int):
+    def step_layers(self, first: int, last: int, bufs=None):
+        """Layers [first, last) of a step; `bufs` (an InputSet) replaces the
+        step's inputs and outputs (q, k_new, v_new, out and the metadata)."""
         pk, w = self.pk, self.w
+        b = bufs or self
         for l in range(first, last):
             c = l % self.ncache
-            if self.pairs is not None:
-                pk.copy_blocks(self.kc[c], self.vc[c], self.pairs, stream=self.stream)
-            pk.reshape_and_cache(self.k_new[l], self.v_new[l], self.kc[c], self.vc[c], self.slots,
+            if b.pairs is not None:
+                pk.copy_blocks(self.kc[c], self.vc[c], b.pairs, stream=self.stream)
+            pk.reshape_and_cache(b.k_new[l], b.v_new[l], self.kc[c], self.vc[c], b.slots,
                                  stream=self.stream)
-            pk.decode(self.out[l], self.q[l], self.kc[c], self.vc[c], self.tables, self.lens,
+            pk.decode(b.out[l], b.q[l], self.kc[c], self.vc[c], b.tables, b.lens,
                       w.num_kv_heads, w.scale, workspace=self.ws, stream=self.stream)
 
     def decode_all(self):
@@ -509,115 +512,119 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(st, args, device, world, chunks: int = 4):
+class InputSet:
+    """One device copy of a step's inputs (q, new k / v, tables, lengths,
+    slots, copy pairs) and outputs."""
+
+    def __init__(self, st, clone: bool):
+        f = (lambda t: t.clone()) if clone else (lambda t: t)
+        self.q, self.k_new, self.v_new, self.out = f(st.q), f(st.k_new), f(st.v_new), f(st.out)
+        self.tables, self.lens, self.slots = f(st.tables), f(st.lens), f(st.slots)
+        self.pairs = f(st.pairs) if st.pairs is not None else None
+
+    def meta(self):
+        return [t for t in (self.tables, self.lens, self.slots, self.pairs) if t is not None]
+
+
+def run_e2e(st, args, device, world, first_groups: int = 4):
     """Same steps, with every step's inputs copied from pinned host memory and
-    its outputs read back, inside the timed region.  Upload and read-back
-    streams move the inputs of the next group of layers while the current
-    group computes and read each group's outputs back as soon as they are
-    done; per-group events keep a step's copies from overwriting buffers the
-    previous step still uses, so copies of one step overlap the compute of
-    its neighbours.  The region ends once the last step's outputs are on the
-    host."""
+    its outputs read back, inside the timed region.
+
+    Steps are double-buffered: two device copies of the inputs and outputs
+    alternate, so step i + 1's upload (its own stream) runs while step i
+    computes, and step i's read-back (a third stream) runs while step i + 1
+    computes.  The compute stream waits on one event per step, so the step's
+    32 layers stay chained by programmatic dependent launch.  An upload into
+    a buffer set waits until the step two back has finished reading it, and a
+    step waits until the read-back two back has finished with its output set.
+    The first timed step has nothing to hide its upload behind, so it is
+    uploaded in layer groups that its compute follows group by group.  The
+    region starts before the first upload and ends when the last step's
+    outputs are on the host."""
     import torch
     L = st.layers
-    per = (L + chunks - 1) // chunks
-    groups = [(c * per, min(L, (c + 1) * per)) for c in range(chunks) if c * per < L]
+    sets = [InputSet(st, clone=False), InputSet(st, clone=True)]
     hq = st.q.cpu().pin_memory()
     hk = st.k_new.cpu().pin_memory()
     hv = st.v_new.cpu().pin_memory()
-    meta = [(st.tables, st.tables.cpu().pin_memory()), (st.lens, st.lens.cpu().pin_memory()),
-            (st.slots, st.slots.cpu().pin_memory())]
-    if st.pairs is not None:
-        meta.append((st.pairs, st.pairs.cpu().pin_memory()))
-    hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    hmeta = [t.cpu().pin_memory() for t in sets[0].meta()]
+    hout = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(h.numel() * h.element_size() for h in (hq, hk, hv)) + \
-        sum(h.numel() * h.element_size() for _, h in meta)
-    d2h = hout.numel() * hout.element_size()
-    up = torch.cuda.Stream(device)      # inputs of each layer group, host -> device
-    meta_s = torch.cuda.Stream(device)  # the step's tables, lengths and slots
-    down = torch.cuda.Stream(device)    # each group's outputs, device -> host
+        sum(h.numel() * h.element_size() for h in hmeta)
+    d2h = hout[0].numel() * hout[0].element_size()
+    up = torch.cuda.Stream(device)      # a step's inputs, host -> device
+    down = torch.cuda.Stream(device)    # a step's outputs, device -> host
     comp = st.stream
-    ev_in = [torch.cuda.Event() for _ in groups]      # inputs of a group are on the device
-    ev_done = [torch.cuda.Event() for _ in groups]    # a group's compute finished
-    ev_read = [torch.cuda.Event() for _ in groups]    # a group's outputs are back on the host
-    ev_meta = torch.cuda.Event()
-    ev_meta_free = torch.cuda.Event()
-    first = [True]
+    ev_up = [torch.cuda.Event() for _ in range(2)]     # set b's inputs are on the device
+    ev_comp = [torch.cuda.Event() for _ in range(2)]   # the step on set b has computed
+    ev_down = [torch.cuda.Event() for _ in range(2)]   # set b's outputs are on the host
+    used = [False, False]
+    per = (L + first_groups - 1) // first_groups
+    groups = [(c * per, min(L, (c + 1) * per)) for c in range(first_groups) if c * per < L]
+    ev_grp = [torch.cuda.Event() for _ in groups]
 
-    def one_serial():
-        with torch.cuda.stream(comp):
-            for dev, host in meta:
-                dev.copy_(host, non_blocking=True)
-            st.q.copy_(hq, non_blocking=True)
-            st.k_new.copy_(hk, non_blocking=True)
-            st.v_new.copy_(hv, non_blocking=True)
-            st.step()
-            hout.copy_(st.out, non_blocking=True)
-
-    def one_overlapped():
-        # Uploads, metadata and read-backs each have their own stream, so a
-        # group's upload waits only for the previous step's use of the same
-        # group, and nothing but the small metadata copy sits between the
-        # previous step's last layer and this step's first.
-        with torch.cuda.stream(meta_s):
-            if not first[0]:
-                meta_s.wait_event(ev_meta_free)   # previous step no longer reads them
-            for dev, host in meta:
-                dev.copy_(host, non_blocking=True)
-            ev_meta.record(meta_s)
+    def upload(b, grouped):
+        s = sets[b]
         with torch.cuda.stream(up):
-            for c, (a, b) in enumerate(groups):
-                if not first[0]:
-                    up.wait_event(ev_done[c])     # previous step no longer reads them
-                st.q[a:b].copy_(hq[a:b], non_blocking=True)
-                st.k_new[a:b].copy_(hk[a:b], non_blocking=True)
-                st.v_new[a:b].copy_(hv[a:b], non_blocking=True)
-                ev_in[c].record(up)
-        comp.wait_event(ev_meta)
-        for c, (a, b) in enumerate(groups):
-            comp.wait_event(ev_in[c])
-            if not first[0]:
-                comp.wait_event(ev_read[c])       # previous outputs are read back
-            st.step_layers(a, b)
-            ev_done[c].record(comp)
-        ev_meta_free.record(comp)
+            if used[b]:
+                up.wait_event(ev_comp[b])           # the step two back has read set b
+            for dev, host in zip(s.meta(), hmeta):
+                dev.copy_(host, non_blocking=True)
+            for g, (a, e) in enumerate(groups if grouped else [(0, L)]):
+                s.q[a:e].copy_(hq[a:e], non_blocking=True)
+                s.k_new[a:e].copy_(hk[a:e], non_blocking=True)
+                s.v_new[a:e].copy_(hv[a:e], non_blocking=True)
+                if grouped:
+                    ev_grp[g].record(up)
+            ev_up[b].record(up)
+
+    def compute(b, grouped):
+        s = sets[b]
+        if used[b]:
+            comp.wait_event(ev_down[b])             # the read-back two back has its outputs
+        if grouped:
+            for g, (a, e) in enumerate(groups):
+                comp.wait_event(ev_grp[g])
+                st.step_layers(a, e, s)
+        else:
+            comp.wait_event(ev_up[b])
+            st.step_layers(0, L, s)
+        ev_comp[b].record(comp)
         with torch.cuda.stream(down):
-            for c, (a, b) in enumerate(groups):
-                down.wait_event(ev_done[c])
-                hout[a:b].copy_(st.out[a:b], non_blocking=True)
-                ev_read[c].record(down)
-        first[0] = False
+            down.wait_event(ev_comp[b])
+            hout[b].copy_(s.out, non_blocking=True)
+            ev_down[b].record(down)
+        used[b] = True
 
-    # with one layer group there is nothing to overlap: one stream, no syncs
-    one = one_overlapped if len(groups) > 1 else one_serial
+    def run(n, t0=None):
+        # step i computes on set i % 2 while step i + 1 uploads into the other
+        upload(0, grouped=True)
+        for i in range(n):
+            if i + 1 < n:
+                upload((i + 1) % 2, grouped=False)
+            compute(i % 2, grouped=(i == 0))
+        comp.wait_event(ev_down[(n - 1) % 2])  # the region ends with the last read-back
 
-    def drain():
-        # the timed region ends when the last outputs are back on the host
-        if one is one_overlapped:
-            comp.wait_event(ev_read[-1])
-
-    for _ in range(max(1, args.warmup)):
-        one()
-    drain()
+    run(max(1, args.warmup))
     barrier(device)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(comp)
-    for _ in range(args.steps):
-        one()
-    drain()
+    a.record(up)  # before the first upload
+    run(args.steps)
     b.record(comp)
     torch.cuda.synchronize()
     barrier(device)
     ms = max_over_ranks(a.elapsed_time(b), device)
-    if not torch.equal(hout[-1].to(device), st.out[-1]):
+    last = (args.steps - 1) % 2
+    if not torch.equal(hout[last].to(device), sets[last].out):
         raise RuntimeError("end-to-end outputs read back differ from the device outputs")
     return {"value": round(world * st.S * args.steps / (ms * 1e-3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms / args.steps, 4),
-            "overlap": (f"upload, metadata and read-back streams, {len(groups)} layer groups" if len(groups) > 1
-                        else "none (one layer): copies and kernels on one stream")}
+            "overlap": "double-buffered steps: step i + 1 uploads and step i - 1 reads back "
+                       "while step i computes; the first timed step uploads in "
+                       f"{len(groups)} layer groups"}
 
 
 # ---------------------------------------------------------------- CPU oracle
