@@ -538,9 +538,10 @@ def run_e2e(st, args, device, world, first_groups: int = 4):
     a buffer set waits until the step two back has finished reading it, and a
     step waits until the read-back two back has finished with its output set.
     The first timed step has nothing to hide its upload behind, so it is
-    uploaded in layer groups that its compute follows group by group.  The
-    region starts before the first upload and ends when the last step's
-    outputs are on the host."""
+    uploaded in layer groups that its compute follows group by group.  A
+    one-layer step has nothing to overlap, and there copies and kernels
+    share one stream.  The region starts before the first upload and ends
+    when the last step's outputs are on the host."""
     import torch
     L = st.layers
     sets = [InputSet(st, clone=False), InputSet(st, clone=True)]
@@ -596,7 +597,7 @@ def run_e2e(st, args, device, world, first_groups: int = 4):
             ev_down[b].record(down)
         used[b] = True
 
-    def run(n, t0=None):
+    def run(n):
         # step i computes on set i % 2 while step i + 1 uploads into the other
         upload(0, grouped=True)
         for i in range(n):
@@ -605,26 +606,43 @@ def run_e2e(st, args, device, world, first_groups: int = 4):
             compute(i % 2, grouped=(i == 0))
         comp.wait_event(ev_down[(n - 1) % 2])  # the region ends with the last read-back
 
-    run(max(1, args.warmup))
+    def run_serial(n):
+        # one layer leaves nothing to overlap: cross-stream handshakes would
+        # cost more than they hide, so copies and kernels share one stream
+        s = sets[0]
+        with torch.cuda.stream(comp):
+            for _ in range(n):
+                for dev, host in zip(s.meta(), hmeta):
+                    dev.copy_(host, non_blocking=True)
+                s.q.copy_(hq, non_blocking=True)
+                s.k_new.copy_(hk, non_blocking=True)
+                s.v_new.copy_(hv, non_blocking=True)
+                st.step_layers(0, L, s)
+                hout[0].copy_(s.out, non_blocking=True)
+
+    serial = L == 1
+    step_loop = run_serial if serial else run
+    step_loop(max(1, args.warmup))
     barrier(device)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(up)  # before the first upload
-    run(args.steps)
+    a.record(comp if serial else up)  # before the first upload
+    step_loop(args.steps)
     b.record(comp)
     torch.cuda.synchronize()
     barrier(device)
     ms = max_over_ranks(a.elapsed_time(b), device)
-    last = (args.steps - 1) % 2
+    last = 0 if serial else (args.steps - 1) % 2
     if not torch.equal(hout[last].to(device), sets[last].out):
         raise RuntimeError("end-to-end outputs read back differ from the device outputs")
     return {"value": round(world * st.S * args.steps / (ms * 1e-3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms / args.steps, 4),
-            "overlap": "double-buffered steps: step i + 1 uploads and step i - 1 reads back "
-                       "while step i computes; the first timed step uploads in "
-                       f"{len(groups)} layer groups"}
+            "overlap": ("none (one layer): copies and kernels on one stream" if serial else
+                        "double-buffered steps: step i + 1 uploads and step i - 1 reads back "
+                        "while step i computes; the first timed step uploads in "
+                        f"{len(groups)} layer groups")}
 
 
 # ---------------------------------------------------------------- CPU oracle
