@@ -377,9 +377,11 @@ __global__ void __launch_bounds__(NW * 32)
 // NT = number of 8-head column tiles (G <= 8 * NT).  With NT == 1 the kernel
 // is compiled for PA_DECODE_MIN_CTAS resident CTAs per SM (80 registers at
 // 6): resident warps, not pipeline depth, set the bandwidth this kernel
-// reaches.
+// reaches.  The 16-head variant holds twice the accumulators; it is
+// compiled for 3 CTAs per SM (at most 168 registers), which it reaches
+// without spilling.
 template <typename T, int D, int NW, int STAGES, int NT, int PB>
-__global__ void __launch_bounds__(NW * 32, NT == 1 ? PA_DECODE_MIN_CTAS : 1)
+__global__ void __launch_bounds__(NW * 32, NT == 1 ? PA_DECODE_MIN_CTAS : 3)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a) {
     using Pipe = WarpPipe<D, STAGES>;
