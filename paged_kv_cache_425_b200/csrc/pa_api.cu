@@ -132,47 +132,80 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
                : PA_ERR_CUDA;
 }
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (ids are never reused
+// within a process, unlike context handles), or 0 when there is none yet or
+// the driver cannot say.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
 // Raise a kernel's dynamic shared-memory limit to `bytes` (once per kernel,
-// device and size: the attribute persists in the context).
+// device, CUDA context and size: the attribute persists in the context, and a
+// device reset starts a new one).
 template <typename Kernel>
 bool set_smem(Kernel k, int bytes) {
     struct Key {
         const void *fn;
         int dev, bytes;
+        unsigned long long ctx;
     };
     static std::mutex mu;
     static std::vector<Key> done;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const unsigned long long ctx = current_context_id();
     const void *fn = reinterpret_cast<const void *>(k);
     std::lock_guard<std::mutex> lock(mu);
     for (const Key &e : done)
-        if (e.fn == fn && e.dev == dev && e.bytes >= bytes) return true;
+        if (ctx != 0 && e.fn == fn && e.dev == dev && e.ctx == ctx && e.bytes >= bytes) return true;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return false;
-    done.push_back({fn, dev, bytes});
+    if (ctx != 0) done.push_back({fn, dev, bytes, ctx});
     return true;
 }
 
 // Registers per thread a kernel was compiled with (-1 on failure); looked up
-// once per kernel and device.
+// once per kernel, device and CUDA context.
 template <typename Kernel>
 int compiled_registers(Kernel k) {
     struct Entry {
         const void *fn;
         int dev, regs;
+        unsigned long long ctx;
     };
     static std::mutex mu;
     static std::vector<Entry> seen;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    const unsigned long long ctx = current_context_id();
     const void *fn = reinterpret_cast<const void *>(k);
     std::lock_guard<std::mutex> lock(mu);
     for (const Entry &e : seen)
-        if (e.fn == fn && e.dev == dev) return e.regs;
+        if (ctx != 0 && e.fn == fn && e.dev == dev && e.ctx == ctx) return e.regs;
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return -1;
-    seen.push_back({fn, dev, fa.numRegs});
+    if (ctx != 0) seen.push_back({fn, dev, fa.numRegs, ctx});
     return fa.numRegs;
 }
 
@@ -672,34 +705,6 @@ struct StaticAddress {
     unsigned long long ctx_id;  // the context the address belongs to
 };
 StaticAddress g_static_address[kMaxDevices] = {};
-
-using CtxGetCurrentFn = CUresult (*)(CUcontext *);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
-
-// Unique id of the calling thread's current context (ids are never reused
-// within a process, unlike context handles), or 0 when there is none yet or
-// the driver cannot say.
-unsigned long long current_context_id() {
-    static CtxGetCurrentFn get_current = nullptr;
-    static CtxGetIdFn get_id = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_id = reinterpret_cast<CtxGetIdFn>(p);
-    });
-    CUcontext ctx = nullptr;
-    unsigned long long id = 0;
-    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
-        get_id(ctx, &id) != CUDA_SUCCESS)
-        return 0;
-    return id;
-}
 
 // Device address of the array in the current device's current context.  A
 // device reset (cudaDeviceReset) ends the context the cached address belongs
