@@ -190,7 +190,7 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
  *
  *   PA_PREFILL_AUTO     the tcgen05 kernel when its conditions hold (q and
  *                       out 16-byte aligned, query group <= 128, scale > 0,
- *                       max_blocks_per_seq <= 8448 at head_dim 128), otherwise
+ *                       max_blocks_per_seq <= 8192 at head_dim 128), otherwise
  *                       the mma.sync kernel.  The default.
  *   PA_PREFILL_MMA_SYNC always the mma.sync kernel (64 packed query rows per
  *                       CTA, warp-level tensor-core tiles, registers hold S).
