@@ -98,8 +98,9 @@ def test_tables_at_the_wide_partition_threshold(hq, hkv, dtype):
 @pytest.mark.parametrize("hq,hkv,dtype", [(4, 4, wl.F16), (8, 2, wl.BF16), (16, 1, wl.BF16)])
 def test_two_eight_and_nine_partitions(hq, hkv, dtype):
     """Tables of 33, 256 and 257 blocks split a context into up to 2, 8 and 9
-    partitions of 512 tokens.  Contexts cover one partition, the partition
-    boundaries, and the whole table."""
+    partitions of 512 tokens: the merge kernel loads all of a row's partials
+    at once up to 8 partitions and loops over them beyond.  Contexts cover
+    one partition, the partition boundaries, and the whole table."""
     for width in (33, 256, 257):
         rng = wl.rng_for(40 + width)
         cap = width * 16
