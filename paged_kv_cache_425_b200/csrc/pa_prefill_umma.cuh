@@ -464,13 +464,28 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             if (__all_sync(FULL, ok)) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
+                const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;
                 uint16_t *orow = reinterpret_cast<uint16_t *>(a.out) +
                                  ((size_t)(q0 + qi) * a.num_q_heads + (size_t)kvh * G + qh) * D;
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 64) {
                     uint32_t o[64];
                     tmem_ld64(t_o + c0, o);
-                    if (rvalid) {
+                    if (rvalid && out32) {
+                        // 32-byte stores: a warp's store covers whole sectors of its
+                        // 32 rows, half as many memory transactions as 16-byte ones
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                w[i] = Mma<T>::pack(__uint_as_float(o[16 * u + 2 * i]) * inv,
+                                                    __uint_as_float(o[16 * u + 2 * i + 1]) * inv);
+                            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(orow + c0 + 16 * u),
+                                         "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                                         : "memory");
+                        }
+                    } else if (rvalid) {
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
                             uint4 v;

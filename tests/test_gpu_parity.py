@@ -569,6 +569,35 @@ def test_prefill_bad_block_id_is_reported(prefill_kernel):
     assert gh.max_excess(out[64:], ref, wl.BF16) <= gh.TOL[wl.BF16]
 
 
+def test_prefill_output_aligned_to_16_bytes_only(prefill_kernel):
+    """q and out start 16 bytes into their buffers: 16-byte aligned, not
+    32.  The tcgen05 kernel then stores its rows in 16-byte pieces instead
+    of 32-byte ones; results are the same, and nothing around out changes."""
+    rng = wl.rng_for(48)
+    lens = np.array([300, 77, 1000], np.int32)
+    qlens = np.array([300, 50, 129], np.int32)
+    hq, hkv, d = 16, 4, 128
+    p = make_paged(rng, 3, hq, hkv, d, lens, wl.blocks_needed(lens, 16) + 2, wl.BF16)
+    T = int(qlens.sum())
+    qchunk = wl.draw_values(rng, (T, hq, d), wl.BF16)
+    n = T * hq * d
+    qbuf = torch.zeros(n + 16, dtype=torch.bfloat16, device="cuda")
+    qbuf[8:8 + n] = gh.to_dev(qchunk, wl.BF16).reshape(-1)
+    obuf = torch.full((n + 16,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    q, out = qbuf[8:8 + n].view(T, hq, d), obuf[8:8 + n].view(T, hq, d)
+    assert out.data_ptr() % 16 == 0 and out.data_ptr() % 32 != 0
+    qs = np.zeros(4, np.int32)
+    qs[1:] = np.cumsum(qlens)
+    pk.prefill(out, q, gh.to_dev(p.key_cache, wl.BF16), gh.to_dev(p.value_cache, wl.BF16),
+               gh.ints(p.tables), gh.ints(p.lens), gh.ints(qs), int(qlens.max()), hkv, p.scale)
+    torch.cuda.synchronize()
+    assert pk.get_error() == (0, 0)
+    ref = oracle.prefill(qchunk, p.key_cache, p.value_cache, p.tables, p.lens, qs, hkv,
+                         p.scale, wl.BF16)
+    assert gh.max_excess(out, ref, wl.BF16) <= gh.TOL[wl.BF16]
+    assert torch.isnan(obuf[:8]).all() and torch.isnan(obuf[8 + n:]).all()
+
+
 @pytest.mark.parametrize("num_seqs", [40, 300])
 def test_prefill_many_sequences_with_equal_lengths(num_seqs, prefill_kernel):
     """Many sequences, lengths repeating (ties in the longest-first CTA
