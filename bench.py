@@ -4,8 +4,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = one decode step of a batch: for every layer, pa_copy_blocks of
-the copy-on-write pairs (parallel-sampling workload only), pa_reshape_and_cache
-of one new token per sequence, then pa_decode over the whole paged context.
+the copy-on-write pairs (parallel-sampling workload only), then
+pa_decode_append, which writes each sequence's new token into its cache slot
+and attends over the whole paged context in one launch (`--step separate`:
+pa_reshape_and_cache, then pa_decode, as two launches; the default run
+measures that form too, under `also_measured`).
 Inputs are resident in HBM before the timed region; each layer has its own
 KV cache (all larger than the 126 MB L2, so no flush is needed).  Prints one
 JSON line: tokens/s (`value`), the decode call's achieved HBM GB/s against
@@ -60,6 +63,9 @@ def parse_args(argv=None):
     ap.add_argument("--prefill-kernel", choices=["auto", "mma_sync", "tcgen05"], default="auto",
                     help="prefill workload: which pa_prefill kernel runs (auto = tcgen05)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--step", choices=["fused", "separate"], default="fused",
+                    help="fused: pa_decode_append per layer; separate: pa_reshape_and_cache "
+                         "then pa_decode")
     ap.add_argument("--extra", default=None,
                     help="comma-separated workloads measured after the main one in the same run "
                          "(default for llama7b: gqa_long,llama13b; 'none' for none); each is "
@@ -100,15 +106,19 @@ def barrier(device=None):
 
 
 # ---------------------------------------------------------------- workload description
-def algorithmic_bytes(lens, num_q_heads, num_kv_heads, head_dim, elem=2, block=16) -> int:
+def algorithmic_bytes(lens, num_q_heads, num_kv_heads, head_dim, elem=2, block=16,
+                      append: bool = False) -> int:
     """Bytes one pa_decode call must move: K and V of every cached token, q and
-    out, the block-table entries it reads and the context lengths."""
+    out, the block-table entries it reads and the context lengths.  With
+    `append` (pa_decode_append): also each sequence's new K and V rows, read
+    once and written once into the cache."""
     lens = np.asarray(lens, dtype=np.int64)
     S = len(lens)
     kv = int(2 * lens.sum() * num_kv_heads * head_dim * elem)
     qo = 2 * S * num_q_heads * head_dim * elem
     tables = int(4 * ((lens + block - 1) // block).sum())
-    return kv + qo + tables + 4 * S
+    new_rows = 2 * 2 * int((lens > 0).sum()) * num_kv_heads * head_dim * elem if append else 0
+    return kv + qo + tables + 4 * S + new_rows
 
 
 # Layer caches allocated per workload when the bench measures it after the
@@ -323,11 +333,20 @@ class Setup:
         self.parts = decode_partitions(b.max_blocks)
         torch.cuda.synchronize(device)
         self.stream = torch.cuda.Stream(device)  # a dedicated stream for every timed call
-        self.bytes_per_call = algorithmic_bytes(b.context_lens, Hq, H, d)
+        self.set_mode(getattr(args, "step", "fused"))
         # K/V bytes of distinct physical blocks (shared prompt blocks once)
         self.unique_kv_bytes = int(b.alloc.stats()["filled_slots"]) * H * d * 2 * 2
-        self.launches_per_step = L * (1 + 1 + (1 if self.parts > 1 else 0)
-                                      + (1 if self.pairs is not None else 0))
+
+    def set_mode(self, mode: str):
+        """fused: pa_decode_append per layer; separate: pa_reshape_and_cache
+        then pa_decode."""
+        b, w = self.batch, self.w
+        self.fused = mode == "fused"
+        self.bytes_per_call = algorithmic_bytes(b.context_lens, w.num_q_heads, w.num_kv_heads,
+                                                w.head_dim, append=self.fused)
+        self.launches_per_step = self.layers * ((1 if self.fused else 2)
+                                                + (1 if self.parts > 1 else 0)
+                                                + (1 if self.pairs is not None else 0))
 
     def step(self):
         self.step_layers(0, self.layers)
@@ -341,18 +360,31 @@ class Setup:
             c = l % self.ncache
             if b.pairs is not None:
                 pk.copy_blocks(self.kc[c], self.vc[c], b.pairs, stream=self.stream)
-            pk.reshape_and_cache(b.k_new[l], b.v_new[l], self.kc[c], self.vc[c], b.slots,
-                                 stream=self.stream)
-            pk.decode(b.out[l], b.q[l], self.kc[c], self.vc[c], b.tables, b.lens,
-                      w.num_kv_heads, w.scale, workspace=self.ws, stream=self.stream)
+            if self.fused:
+                pk.decode_append(b.out[l], b.q[l], b.k_new[l], b.v_new[l], self.kc[c],
+                                 self.vc[c], b.tables, b.lens, w.num_kv_heads, w.scale,
+                                 workspace=self.ws, stream=self.stream)
+            else:
+                pk.reshape_and_cache(b.k_new[l], b.v_new[l], self.kc[c], self.vc[c], b.slots,
+                                     stream=self.stream)
+                pk.decode(b.out[l], b.q[l], self.kc[c], self.vc[c], b.tables, b.lens,
+                          w.num_kv_heads, w.scale, workspace=self.ws, stream=self.stream)
 
     def decode_all(self):
-        """Only the decode calls of one step (every layer's own cache)."""
+        """Only the attention calls of one step (every layer's own cache):
+        pa_decode_append in the fused mode (writing the same rows again),
+        pa_decode otherwise."""
         pk, w = self.pk, self.w
         for l in range(self.layers):
             c = l % self.ncache
-            pk.decode(self.out[l], self.q[l], self.kc[c], self.vc[c], self.tables, self.lens,
-                      w.num_kv_heads, w.scale, workspace=self.ws, stream=self.stream)
+            if self.fused:
+                pk.decode_append(self.out[l], self.q[l], self.k_new[l], self.v_new[l],
+                                 self.kc[c], self.vc[c], self.tables, self.lens, w.num_kv_heads,
+                                 w.scale, workspace=self.ws, stream=self.stream)
+            else:
+                pk.decode(self.out[l], self.q[l], self.kc[c], self.vc[c], self.tables,
+                          self.lens, w.num_kv_heads, w.scale, workspace=self.ws,
+                          stream=self.stream)
 
 
 def measure(st, args, device, world) -> dict:
@@ -407,10 +439,17 @@ def roofline_record(st, workload: str, dec_avg_ms: float) -> dict:
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": traffic_per_call(workload, st.bytes_per_call),
-            "kernel": "pa_decode call (partition kernel + merge kernel), timed over the "
-                      "step's layer calls run back to back",
+            "kernel": ("pa_decode_append call (new-row write + partition kernel + merge kernel)"
+                       if st.fused else "pa_decode call (partition kernel + merge kernel)")
+                      + ", timed over the step's layer calls run back to back",
             "algorithmic_bytes_per_call": st.bytes_per_call,
             "avg_call_us": round(dec_avg_ms * 1e3, 2), "peak_source": peak_src}
+
+
+def step_calls(st) -> str:
+    """The library calls one layer of the step makes."""
+    calls = "pa_decode_append" if st.fused else "pa_reshape_and_cache, pa_decode"
+    return ("pa_copy_blocks, " if st.pairs is not None else "") + calls + " per layer"
 
 
 def extra_workloads(args) -> list:
@@ -440,7 +479,25 @@ def run_ours(args, world, rank, local):
     main = {"w": st.w, "lens": st.batch.context_lens, "nb": st.nb, "max_blocks": st.batch.max_blocks,
             "S": st.S, "ncache": st.ncache, "alloc_seconds": st.alloc_seconds,
             "unique_kv_bytes": st.unique_kv_bytes, "launches": st.launches_per_step,
-            "roofline": roofline_record(st, args.workload, dec_avg_ms)}
+            "roofline": roofline_record(st, args.workload, dec_avg_ms),
+            "step": step_calls(st)}
+    # ---- the default run also times the two-launch step on the same inputs
+    separate = None
+    if st.fused and extra_workloads(args):
+        st.set_mode("separate")
+        ms = measure(st, args, device, world)
+        separate = {
+            "value": round(world * st.S * args.steps / (ms["total_ms"] * 1e-3), 1),
+            "unit": "tokens/s",
+            "ms_per_step": round(ms["total_ms"] / args.steps, 4),
+            "ms_per_step_p10_p50_p90": [round(float(np.percentile(ms["step_ms"], q)), 4)
+                                        for q in (10, 50, 90)],
+            "step": step_calls(st),
+            "config": describe(st.w, st.batch.context_lens, st.nb, st.batch.max_blocks, world),
+            "roofline": roofline_record(st, args.workload, ms["dec_avg_ms"]),
+            "gpu_launches": st.launches_per_step * args.steps,
+            "clocks": ms["clocks"],
+        }
     del st
     torch.cuda.empty_cache()
 
@@ -455,6 +512,7 @@ def run_ours(args, world, rank, local):
             "value": round(world * sx.S * args.steps / (mx["total_ms"] * 1e-3), 1),
             "unit": "tokens/s",
             "ms_per_step": round(mx["total_ms"] / args.steps, 4),
+            "step": step_calls(sx),
             "ms_per_step_p10_p50_p90": [round(float(np.percentile(mx["step_ms"], q)), 4)
                                         for q in (10, 50, 90)],
             "dtype": "f16" if sx.w.dtype == wl.F16 else "bf16",
@@ -466,6 +524,8 @@ def run_ours(args, world, rank, local):
         }
         del sx
         torch.cuda.empty_cache()
+    if separate is not None:
+        subs[f"{args.workload}_separate_calls"] = separate
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -494,6 +554,7 @@ def run_ours(args, world, rank, local):
         "dtype": "f16" if w.dtype == wl.F16 else "bf16",
         "data": "synthetic: seeded N(0,1) q/k/v/cache, seeded context lengths, allocator-built scattered tables",
         "config": describe(w, main["lens"], main["nb"], main["max_blocks"], world),
+        "step": main["step"],
         "layer_caches": main["ncache"],
         "unique_kv_bytes_per_call": main["unique_kv_bytes"],
         "host_alloc_seconds": round(main["alloc_seconds"], 3),

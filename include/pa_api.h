@@ -156,6 +156,38 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * pa_decode_append - write each sequence's new token into the cache, then
+ * decode: pa_reshape_and_cache followed by pa_decode, in one launch.
+ *
+ * Source: the passages of pa_reshape_and_cache and pa_decode.  A decode step
+ * appends one token per sequence at position L - 1 (L = context_lens[s],
+ * the new token included) and attends over all L tokens; this call does
+ * both, so the step needs no separate write launch.
+ *
+ * Equivalent to pa_reshape_and_cache(k_new, v_new, ..., slot_mapping) with
+ * slot_mapping[s] = block_tables[s][(L - 1) / 16] * 16 + (L - 1) % 16,
+ * followed by pa_decode(...) with the same arguments: the same cache bytes
+ * afterwards, and the same outputs, bit for bit.  Sequences with L == 0
+ * write nothing (zero output row).  An out-of-range block id at position
+ * L - 1 writes nothing and sets PA_DEVERR_BLOCK_ID, as pa_decode reports it.
+ * The block holding position L - 1 must belong to this sequence alone (the
+ * allocator copies a shared last block before appending to it): another
+ * sequence that reads it in the same call may see the slot before or after
+ * the write.  Argument checks, workspace and errors are those of pa_decode.
+ *
+ *   k_new, v_new  device, [num_seqs][num_kv_heads][head_dim], dtype,
+ *                 contiguous, 16-byte aligned (PA_ERR_INVALID_ARG otherwise)
+ *   key_cache,    device, cache layout of pa_decode (one row per sequence and
+ *   value_cache   kv head written, the rest read)
+ */
+int pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                     void *key_cache, void *value_cache, const int32_t *block_tables,
+                     const int32_t *context_lens, int32_t num_kv_heads, float scale,
+                     int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t block_size,
+                     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * pa_prefill - chunked-prefill attention over the paged cache.
  *
  * Source: "PagedAttention in vLLM: a throughput settings guide", section

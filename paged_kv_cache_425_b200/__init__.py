@@ -76,6 +76,8 @@ pa_reshape_and_cache = _sig("pa_reshape_and_cache", ctypes.c_int, _P, _P, _P, _P
                             _i32, _i32, _i64, _i32, _P)
 pa_decode = _sig("pa_decode", ctypes.c_int, _P, _P, _P, _P, _P, _P, _i32, _f32, _i32, _i32, _i32,
                  _i32, _i32, _i64, _i32, _P, _sz, _P)
+pa_decode_append = _sig("pa_decode_append", ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _i32,
+                        _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P, _sz, _P)
 pa_decode_workspace_size = _sig("pa_decode_workspace_size", _sz, _i32, _i32, _i32, _i32, _i32)
 pa_decode_static_workspace = _sig("pa_decode_static_workspace", ctypes.c_int, _P, _P, _P, _P, _P,
                                   _P, _i32, _f32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P)
@@ -208,6 +210,38 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, num_kv_he
                      _dev(context_lens, "context_lens", torch.int32, 1), hkv, float(scale), S, hq,
                      d, bs, maxb, nb, dtype_code(q), ws_ptr, ws_bytes, _stream(stream)),
            "pa_decode")
+
+
+def decode_append(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens,
+                  num_kv_heads: int, scale: float, workspace=None, stream=None):
+    """Write each sequence's new token (k_new, v_new: [S, Hkv, d]) at position
+    context_lens[s] - 1 of its table, then decode, in one launch: the same
+    cache bytes and outputs as reshape_and_cache followed by decode."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_shape(key_cache, value_cache)
+    if hkv != num_kv_heads:
+        raise ValueError("num_kv_heads does not match the cache")
+    S, hq, dq = q.shape
+    if dq != d or tuple(out.shape) != (S, hq, d) or out.dtype != q.dtype or q.dtype != key_cache.dtype:
+        raise ValueError("q / out must be [S, Hq, d] of the cache dtype")
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if tuple(t.shape) != (S, hkv, d) or t.dtype != key_cache.dtype:
+            raise ValueError(f"{name} must be [S, Hkv, d] of the cache dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    maxb = int(block_tables.shape[1])
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(pa_decode_append(_dev(out, "out"), _dev(q, "q"), _dev(k_new, "k_new"),
+                            _dev(v_new, "v_new"), _dev(key_cache, "key_cache"),
+                            _dev(value_cache, "value_cache"),
+                            _dev(block_tables, "block_tables", torch.int32, 2),
+                            _dev(context_lens, "context_lens", torch.int32, 1), hkv, float(scale),
+                            S, hq, d, bs, maxb, nb, dtype_code(q), ws_ptr, ws_bytes,
+                            _stream(stream)),
+           "pa_decode_append")
 
 
 def prefill(out, q, key_cache, value_cache, block_tables, context_lens, query_start,

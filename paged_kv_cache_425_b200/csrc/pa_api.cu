@@ -430,21 +430,15 @@ int check_decode_args(const void *out, const void *q, const void *key_cache,
     if (num_parts_for(max_blocks_per_seq) > 8192) return PA_ERR_UNSUPPORTED;
     return PA_OK;
 }
-}  // namespace
-}  // namespace pa
 
-extern "C" {
-
-int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
-              const int32_t *block_tables, const int32_t *context_lens, int32_t num_kv_heads,
-              float scale, int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
-              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
-              void *workspace, size_t workspace_bytes, void *stream) {
-    bool empty = false;
-    const int rc = check_decode_args(out, q, key_cache, value_cache, block_tables, context_lens,
-                                     num_kv_heads, num_seqs, num_q_heads, head_dim, block_size,
-                                     max_blocks_per_seq, num_blocks, dtype, &empty);
-    if (rc != PA_OK || empty) return rc;
+// pa_decode, and pa_decode_append when k_new / v_new are given (arguments
+// already checked, at least one sequence).
+int decode_call(void *out, const void *q, const void *k_new, const void *v_new, void *key_cache,
+                void *value_cache, const int32_t *block_tables, const int32_t *context_lens,
+                int32_t num_kv_heads, float scale, int32_t num_seqs, int32_t num_q_heads,
+                int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                int64_t num_blocks, int32_t dtype, void *workspace, size_t workspace_bytes,
+                void *stream) {
     const int group = num_q_heads / num_kv_heads;
     const int64_t parts = num_parts_for(max_blocks_per_seq);
 
@@ -463,6 +457,10 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.num_parts = (int)parts;
     a.part_blocks = part_blocks_for(max_blocks_per_seq);
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.key_cache = key_cache;
+    a.value_cache = value_cache;
     if (parts > 1) {
         const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, block_size,
                                                      max_blocks_per_seq);
@@ -480,6 +478,43 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return dtype == PA_F16 ? dispatch_decode<__half>(a, head_dim, group, tmk, tmv, st)
                            : dispatch_decode<__nv_bfloat16>(a, head_dim, group, tmk, tmv, st);
+}
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *context_lens, int32_t num_kv_heads,
+              float scale, int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
+              void *workspace, size_t workspace_bytes, void *stream) {
+    bool empty = false;
+    const int rc = check_decode_args(out, q, key_cache, value_cache, block_tables, context_lens,
+                                     num_kv_heads, num_seqs, num_q_heads, head_dim, block_size,
+                                     max_blocks_per_seq, num_blocks, dtype, &empty);
+    if (rc != PA_OK || empty) return rc;
+    return decode_call(out, q, nullptr, nullptr, const_cast<void *>(key_cache),
+                       const_cast<void *>(value_cache), block_tables, context_lens, num_kv_heads,
+                       scale, num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                       num_blocks, dtype, workspace, workspace_bytes, stream);
+}
+
+int pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                     void *key_cache, void *value_cache, const int32_t *block_tables,
+                     const int32_t *context_lens, int32_t num_kv_heads, float scale,
+                     int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t block_size,
+                     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t dtype,
+                     void *workspace, size_t workspace_bytes, void *stream) {
+    bool empty = false;
+    const int rc = check_decode_args(out, q, key_cache, value_cache, block_tables, context_lens,
+                                     num_kv_heads, num_seqs, num_q_heads, head_dim, block_size,
+                                     max_blocks_per_seq, num_blocks, dtype, &empty);
+    if (rc != PA_OK || empty) return rc;
+    if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return PA_ERR_INVALID_ARG;
+    return decode_call(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens,
+                       num_kv_heads, scale, num_seqs, num_q_heads, head_dim, block_size,
+                       max_blocks_per_seq, num_blocks, dtype, workspace, workspace_bytes, stream);
 }
 
 int pa_prefill_select(int32_t kernel) {

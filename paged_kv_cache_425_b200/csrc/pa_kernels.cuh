@@ -65,6 +65,12 @@ struct DecodeArgs {
     int part_blocks;   // blocks per partition for this call (the decode kernels
                        // also take it as their PB template argument)
     float scale_log2;  // scale * log2(e)
+    // pa_decode_append only (null otherwise): each sequence's new token,
+    // [S][Hkv][D], written into the caches at position L - 1 before it is read
+    const void *k_new;
+    const void *v_new;
+    void *key_cache;
+    void *value_cache;
 };
 
 __device__ __forceinline__ int clamp_context(const DecodeArgs &a, int s, bool report) {
@@ -182,6 +188,45 @@ __device__ __forceinline__ int warp_block_count(int nb_local, int warp, int nw) 
     return warp < nb_local ? (nb_local - warp + nw - 1) / nw : 0;
 }
 
+// pa_decode_append: the warp whose blocks include the one holding position
+// L - 1 writes sequence s's new K and V rows for kv head kvh into that slot
+// before it issues that block's load.  Each writing lane orders its store
+// before the async-proxy (TMA) reads with a proxy fence; the warp then syncs,
+// and lane 0 issues the loads.  Other warps and CTAs never read that slot in
+// this call (partitions are disjoint token ranges).
+//
+// append_block_index: the warp's own index k of that block (its k-th block
+// is b_begin + warp + k * nw), or -1 when another warp or CTA holds it.
+__device__ __forceinline__ int append_block_index(const DecodeArgs &a, int L, int b_begin,
+                                                  int nb_local, int warp, int nw) {
+    if (a.k_new == nullptr || L <= 0) return -1;
+    const int li = (L - 1) / kBlock - b_begin;
+    if (li < 0 || li >= nb_local || li % nw != warp) return -1;
+    return li / nw;
+}
+
+// The write itself (whole warp).  A bad block id is reported where the block
+// is loaded; nothing is written then.
+template <int D>
+__device__ __forceinline__ void append_new_token(const DecodeArgs &a, int s, int kvh, int L,
+                                                 int lane) {
+    const int phys = a.block_tables[(size_t)s * a.max_blocks_per_seq + (L - 1) / kBlock];
+    if (phys < 0 || phys >= a.num_blocks) return;  // the same for the whole warp
+    constexpr int U = D / 8;  // 16-byte units per row: lanes 0..U-1 copy K, U..2U-1 copy V
+    if (lane < 2 * U) {
+        const bool is_v = lane >= U;
+        const int u = is_v ? lane - U : lane;
+        const size_t src = ((size_t)s * a.num_kv_heads + kvh) * D + (size_t)u * 8;
+        const size_t dst =
+            (((size_t)phys * a.num_kv_heads + kvh) * kBlock + (L - 1) % kBlock) * D + (size_t)u * 8;
+        const uint4 v =
+            *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(is_v ? a.v_new : a.k_new) + src);
+        *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(is_v ? a.value_cache : a.key_cache) + dst) = v;
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    __syncwarp();
+}
+
 // ------------------------------------------------------------------ decode: one q head per kv head
 template <typename T, int D, int NW, int STAGES, int PB>
 __global__ void __launch_bounds__(NW * 32)
@@ -239,7 +284,13 @@ __global__ void __launch_bounds__(NW * 32)
     }
     __syncwarp();
     int issued = nk < STAGES ? nk : STAGES;
+    // pa_decode_append: write the new token before the load of its block; if
+    // that load is not among the first ones, after them, so that the write's
+    // latency overlaps theirs
+    const int k_app = append_block_index(a, L, b_begin, nb_local, warp, NW);
+    if (k_app >= 0 && k_app < issued) append_new_token<D>(a, s, kvh, L, lane);
     for (int k = 0; k < issued; ++k) pipe.issue(k);
+    if (k_app >= issued) append_new_token<D>(a, s, kvh, L, lane);
 
     float qv[EPL];
     {
@@ -436,7 +487,13 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? PA_DECODE_MIN_CTAS : 3)
     }
     __syncwarp();
     int issued = nk < STAGES ? nk : STAGES;
+    // pa_decode_append: write the new token before the load of its block; if
+    // that load is not among the first ones, after them, so that the write's
+    // latency overlaps theirs
+    const int k_app = append_block_index(a, L, b_begin, nb_local, warp, NW);
+    if (k_app >= 0 && k_app < issued) append_new_token<D>(a, s, kvh, L, lane);
     for (int k = 0; k < issued; ++k) pipe.issue(k);
+    if (k_app >= issued) append_new_token<D>(a, s, kvh, L, lane);
 
     const int g = lane >> 2, c = lane & 3;
     // B operand of S^T = K Q^T: lane holds Q[h = 8 nt + g][16 kk + 2c .. +1] and [.. + 8 ..].

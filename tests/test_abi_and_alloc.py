@@ -495,6 +495,32 @@ def test_static_workspace_decode_checks_arguments_like_pa_decode():
     assert a == b == pk.PA_ERR_UNSUPPORTED
 
 
+def test_decode_append_checks_arguments_like_pa_decode():
+    """pa_decode_append applies pa_decode's checks first, then its own on
+    the new rows (present, 16-byte aligned).  Host checks only: every case
+    returns before a launch, and the pointers (aligned placeholders, or
+    none) are never dereferenced."""
+    huge_s, d, maxb, nb = 1 << 20, 128, 4096, 1024
+    for hq, hkv in ((64, 2), (30, 4)):
+        a = pk.pa_decode(None, None, None, None, None, None, hkv, 0.1, huge_s, hq, d, 16, maxb,
+                         nb, pk.F16, None, 0, None)
+        b = pk.pa_decode_append(None, None, None, None, None, None, None, None, hkv, 0.1, huge_s,
+                                hq, d, 16, maxb, nb, pk.F16, None, 0, None)
+        assert a == b and a in (pk.PA_ERR_UNSUPPORTED, pk.PA_ERR_INVALID_ARG), (hq, hkv, a, b)
+    fake = [4096 * (i + 1) for i in range(8)]
+    out, q, kn, vn, kc, vc, tb, ln = fake
+    # no sequences: nothing to do, whatever the new rows are
+    assert pk.pa_decode_append(out, q, None, None, kc, vc, tb, ln, 8, 0.1, 0, 32, d, 16, 64,
+                               nb, pk.BF16, None, 0, None) == pk.PA_OK
+    # missing or misaligned new rows
+    for k_new, v_new in ((None, vn), (kn, None), (kn + 8, vn), (kn, vn + 4)):
+        assert pk.pa_decode_append(out, q, k_new, v_new, kc, vc, tb, ln, 8, 0.1, 4, 32, d, 16,
+                                   64, nb, pk.BF16, None, 0, None) == pk.PA_ERR_INVALID_ARG
+    # a split context without a workspace is refused after the new-row checks pass
+    assert pk.pa_decode_append(out, q, kn, vn, kc, vc, tb, ln, 8, 0.1, 4, 32, d, 16, 64, nb,
+                               pk.BF16, None, 0, None) == pk.PA_ERR_WORKSPACE
+
+
 def test_tcgen05_prefill_refuses_tables_beyond_its_shared_memory():
     """The tcgen05 prefill stages a CTA's block ids in shared memory, beside
     the query tiles and K/V rings, leaving 2 KiB for static shared memory:

@@ -56,6 +56,97 @@ def test_tiny_workload_step():
     assert gh.max_err(out, oracle_out(p)) <= gh.TOL[w.dtype]
 
 
+# ---------------------------------------------------------------- fused append + decode
+def append_slots(p):
+    """Slot of each sequence's last position (its new token), from its table."""
+    return np.array([p.tables[s, (L - 1) // 16] * 16 + (L - 1) % 16 if L > 0 else -1
+                     for s, L in enumerate(p.lens)], np.int64)
+
+
+@pytest.mark.parametrize("hq,hkv,d,dtype", [(4, 4, 64, wl.F16), (32, 32, 128, wl.F16),
+                                            (32, 8, 128, wl.BF16), (16, 1, 128, wl.BF16),
+                                            (12, 1, 64, wl.F16)])
+def test_decode_append_equals_scatter_then_decode(hq, hkv, d, dtype):
+    """pa_decode_append against pa_reshape_and_cache + pa_decode on copies of
+    one pool: the same pool bytes and the same outputs, bit for bit; and both
+    against the oracle's write and attention.  Lengths put the new token
+    first in a block, last in a block, alone in a context, and in the last of
+    several partitions; one sequence is empty."""
+    rng = wl.rng_for(60 + hq + d)
+    lens = np.array([1, 16, 17, 32, 100, 511, 513, 1024, 1025, 3000, 0], np.int32)
+    p = make_paged(rng, len(lens), hq, hkv, d, lens, wl.blocks_needed(lens, 16) + 5, dtype)
+    k_new = wl.draw_values(rng, (len(lens), hkv, d), dtype)
+    v_new = wl.draw_values(rng, (len(lens), hkv, d), dtype)
+    slots = append_slots(p)
+    tbl, ln = gh.ints(p.tables), gh.ints(p.lens)
+    dk, dv = gh.to_dev(k_new, dtype), gh.to_dev(v_new, dtype)
+    q = gh.to_dev(p.q, dtype)
+    ws = gh.workspace_for(pk, len(lens), hq, d, p.tables.shape[1])
+
+    kc1, vc1 = gh.to_dev(p.key_cache, dtype), gh.to_dev(p.value_cache, dtype)
+    out1 = torch.full_like(q, float("nan"))
+    pk.reshape_and_cache(dk, dv, kc1, vc1, gh.ints(slots, torch.int64))
+    pk.decode(out1, q, kc1, vc1, tbl, ln, hkv, p.scale, workspace=ws)
+    kc2, vc2 = gh.to_dev(p.key_cache, dtype), gh.to_dev(p.value_cache, dtype)
+    out2 = torch.full_like(q, float("nan"))
+    pk.decode_append(out2, q, dk, dv, kc2, vc2, tbl, ln, hkv, p.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert pk.get_error() == (0, 0)
+    assert torch.equal(kc1, kc2) and torch.equal(vc1, vc2)
+    assert torch.equal(out1, out2)
+
+    oracle.reshape_and_cache(k_new, v_new, p.key_cache, p.value_cache, slots)
+    assert np.array_equal(gh.to_host_bits(kc2), p.key_cache)
+    assert np.array_equal(gh.to_host_bits(vc2), p.value_cache)
+    assert gh.max_err(out2, oracle_out(p)) <= gh.TOL[dtype]
+
+
+def test_decode_append_bad_last_block_writes_nothing():
+    """An out-of-range id where sequence 1's new token goes: reported as a bad
+    block id, nothing written anywhere, the other sequences exact."""
+    rng = wl.rng_for(66)
+    lens = np.array([40, 70, 300], np.int32)
+    p = make_paged(rng, 3, 8, 2, 128, lens, wl.blocks_needed(lens, 16) + 2, wl.BF16)
+    k_new = wl.draw_values(rng, (3, 2, 128), wl.BF16)
+    v_new = wl.draw_values(rng, (3, 2, 128), wl.BF16)
+    slots = append_slots(p)
+    p.tables[1, (70 - 1) // 16] = p.key_cache.shape[0] + 3
+    kc, vc = gh.to_dev(p.key_cache, wl.BF16), gh.to_dev(p.value_cache, wl.BF16)
+    q = gh.to_dev(p.q, wl.BF16)
+    out = torch.full_like(q, float("nan"))
+    pk.decode_append(out, q, gh.to_dev(k_new, wl.BF16), gh.to_dev(v_new, wl.BF16), kc, vc,
+                     gh.ints(p.tables), gh.ints(p.lens), 2, p.scale)
+    torch.cuda.synchronize()
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_BLOCK_ID
+    slots[1] = -1  # the oracle writes the other two
+    oracle.reshape_and_cache(k_new, v_new, p.key_cache, p.value_cache, slots)
+    assert np.array_equal(gh.to_host_bits(kc), p.key_cache)
+    assert np.array_equal(gh.to_host_bits(vc), p.value_cache)
+    ref = oracle.decode(p.q, p.key_cache, p.value_cache, p.tables, p.lens, 2, p.scale, wl.BF16,
+                        seqs=[0, 2])
+    assert gh.max_err(out[[0, 2]], ref) <= gh.TOL[wl.BF16]
+
+
+def test_decode_append_checks_its_new_rows():
+    rng = wl.rng_for(67)
+    lens = np.array([5, 9], np.int32)
+    p = make_paged(rng, 2, 4, 4, 64, lens, 4, wl.F16)
+    kc, vc = gh.to_dev(p.key_cache, wl.F16), gh.to_dev(p.value_cache, wl.F16)
+    q = gh.to_dev(p.q, wl.F16)
+    out = torch.empty_like(q)
+    kn = torch.zeros((2, 4, 64), dtype=torch.float16, device="cuda")
+    with pytest.raises(ValueError):
+        pk.decode_append(out, q, kn[:, :2], kn, kc, vc, gh.ints(p.tables), gh.ints(p.lens), 4,
+                         p.scale)
+    buf = torch.zeros(2 * 4 * 64 + 4, dtype=torch.float16, device="cuda")
+    misaligned = buf[4:].view(2, 4, 64)  # 8 bytes past a 16-byte boundary
+    with pytest.raises(pk.PagedError) as e:
+        pk.decode_append(out, q, misaligned, kn, kc, vc, gh.ints(p.tables), gh.ints(p.lens), 4,
+                         p.scale)
+    assert e.value.status == pk.PA_ERR_INVALID_ARG
+
+
 # ---------------------------------------------------------------- shapes x lengths
 LENS = [1, 15, 16, 17, 100, 511, 512, 513, 1024, 1500, 2049, 3000]
 
