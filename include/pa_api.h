@@ -221,13 +221,13 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
  * pa_prefill_select - which kernel pa_prefill runs (process-wide).
  *
  *   PA_PREFILL_AUTO     the tcgen05 kernel when its conditions hold (q and
- *                       out 16-byte aligned, query group <= 128, scale > 0,
- *                       max_blocks_per_seq <= 8192 at head_dim 128), otherwise
- *                       the mma.sync kernel.  The default.
+ *                       out 16-byte aligned, query group <= 128, scale > 0),
+ *                       otherwise the mma.sync kernel.  The default.
  *   PA_PREFILL_MMA_SYNC always the mma.sync kernel (64 packed query rows per
  *                       CTA, warp-level tensor-core tiles, registers hold S).
- *   PA_PREFILL_TCGEN05  always the tcgen05 kernel (two tiles of 128 packed
- *                       query rows per CTA, S, P and O in tensor memory); pa_prefill
+ *   PA_PREFILL_TCGEN05  always the tcgen05 kernel (work items of two tiles of
+ *                       128 packed query rows, walked by one persistent CTA
+ *                       per SM; S, P and O in tensor memory); pa_prefill
  *                       returns PA_ERR_UNSUPPORTED when its conditions fail.
  * Both compute the same operation; results differ only by rounding order.
  * Returns PA_OK, or PA_ERR_INVALID_ARG for an unknown value.

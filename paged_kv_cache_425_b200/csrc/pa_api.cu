@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -209,6 +210,22 @@ int compiled_registers(Kernel k) {
     return fa.numRegs;
 }
 
+// Streaming multiprocessors of the current device (-1 on failure); looked up
+// once per device.
+int sm_count() {
+    static std::mutex mu;
+    static std::vector<std::pair<int, int>> seen;  // (device, SMs)
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto &e : seen)
+        if (e.first == dev) return e.second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    seen.push_back({dev, n});
+    return n;
+}
+
 template <typename T, int D, int PB>
 int launch_decode(const DecodeArgs &a, int group, const CUtensorMap &tmk, const CUtensorMap &tmv,
                   cudaStream_t st) {
@@ -303,8 +320,9 @@ WorkspaceLayout workspace_layout(int64_t num_seqs, int64_t num_q_heads, int64_t 
     return l;
 }
 
-// pa_prefill on the tcgen05 kernel: grid x = (sequence, kv head), y = tile of
-// 128 packed query rows (the largest multiple of the group size <= 128).
+// pa_prefill on the tcgen05 kernel: work items of two query tiles of 128
+// packed rows (the largest multiple of the group size <= 128) per (sequence,
+// kv head), walked by one persistent CTA per SM.
 int launch_prefill_umma(void *out, const void *q, const void *key_cache, const void *value_cache,
                         const int32_t *block_tables, const int32_t *context_lens,
                         const int32_t *query_start, int32_t max_query_len, int32_t num_kv_heads,
@@ -335,11 +353,14 @@ int launch_prefill_umma(void *out, const void *q, const void *key_cache, const v
         !encode_cache_map(&tmk, key_cache, num_blocks, num_kv_heads, head_dim, dtype) ||
         !encode_cache_map(&tmv, value_cache, num_blocks, num_kv_heads, head_dim, dtype))
         return PA_ERR_CUDA;
-    const int64_t ctas = (int64_t)num_seqs * num_kv_heads * tiles;
-    if (ctas >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
-    const dim3 grid((unsigned)ctas);
-    const int smem = head_dim == 128 ? prefill_umma_smem_bytes<128>(max_blocks_per_seq)
-                                     : prefill_umma_smem_bytes<64>(max_blocks_per_seq);
+    const int64_t items = (int64_t)num_seqs * num_kv_heads * tiles;
+    if (items >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    // persistent: one CTA per SM (tensor memory and shared memory allow no
+    // second), each walking its share of the items
+    const int sms = sm_count();
+    if (sms <= 0) return PA_ERR_CUDA;
+    const dim3 grid((unsigned)std::min<int64_t>(items, sms));
+    const int smem = head_dim == 128 ? prefill_umma_smem_bytes<128>() : prefill_umma_smem_bytes<64>();
     auto launch = [&](auto kernel) -> int {
         // the kernel re-splits its registers per warpgroup (setmaxnreg); a
         // split above what the launch holds would wait forever, so check the
@@ -547,12 +568,8 @@ int pa_prefill(void *out, const void *q, const void *key_cache, const void *valu
         return PA_ERR_INVALID_ARG;
     if ((int64_t)num_seqs * num_kv_heads >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
     const int which = g_prefill_kernel.load();
-    const int64_t umma_smem = (head_dim == 128 ? prefill_umma_smem_bytes<128>(0)
-                                               : prefill_umma_smem_bytes<64>(0)) +
-                              4 * (int64_t)max_blocks_per_seq;
-    // (227 KiB per CTA covers static shared memory too: leave 2 KiB for it)
     const bool umma_ok = group <= kUmmaRows && aligned(q, 16) && aligned(out, 16) &&
-                         scale > 0.f && scale < 3.0e38f && umma_smem + 2048 <= 227 * 1024;
+                         scale > 0.f && scale < 3.0e38f;
     if (which == PA_PREFILL_TCGEN05 && !umma_ok) return PA_ERR_UNSUPPORTED;
     if (which != PA_PREFILL_MMA_SYNC && umma_ok) {
         const int urc = launch_prefill_umma(out, q, key_cache, value_cache, block_tables,

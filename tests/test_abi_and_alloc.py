@@ -519,18 +519,3 @@ def test_decode_append_checks_arguments_like_pa_decode():
     # a split context without a workspace is refused after the new-row checks pass
     assert pk.pa_decode_append(out, q, kn, vn, kc, vc, tb, ln, 8, 0.1, 4, 32, d, 16, 64, nb,
                                pk.BF16, None, 0, None) == pk.PA_ERR_WORKSPACE
-
-
-def test_tcgen05_prefill_refuses_tables_beyond_its_shared_memory():
-    """The tcgen05 prefill stages a CTA's block ids in shared memory, beside
-    the query tiles and K/V rings, leaving 2 KiB for static shared memory:
-    at head_dim 128 it takes tables of up to 8192 blocks.  Forced onto it, a
-    wider table is refused on the host (the pointers are aligned
-    placeholders; nothing is launched or dereferenced)."""
-    fake = [4096 * (i + 1) for i in range(7)]
-    assert pk.pa_prefill_select(2) == 0  # PA_PREFILL_TCGEN05
-    try:
-        rc = pk.pa_prefill(*fake, 512, 8, 0.1, 1, 32, 512, 128, 16, 8193, 1 << 20, pk.BF16, None)
-        assert rc == pk.PA_ERR_UNSUPPORTED
-    finally:
-        assert pk.pa_prefill_select(0) == 0  # back to PA_PREFILL_AUTO

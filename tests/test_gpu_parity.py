@@ -660,6 +660,22 @@ def test_prefill_bad_block_id_is_reported(prefill_kernel):
     assert gh.max_excess(out[64:], ref, wl.BF16) <= gh.TOL[wl.BF16]
 
 
+def test_prefill_wide_block_tables(prefill_kernel):
+    """Block tables 9000 entries wide (144,000 tokens of room), contexts up to
+    3000 tokens: the tcgen05 kernel reads block ids from the table in global
+    memory, so the width is not limited by shared memory."""
+    rng = wl.rng_for(68)
+    lens = np.array([3000, 700, 129], np.int32)
+    qlens = np.array([200, 64, 129], np.int32)
+    p = make_paged(rng, 3, 16, 4, 128, lens, wl.blocks_needed(lens, 16) + 2, wl.BF16,
+                   max_blocks=9000)
+    assert p.tables.shape == (3, 9000)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), 16, 128), wl.BF16)
+    out, ref = run_prefill(p, qchunk, qlens)
+    assert pk.get_error() == (0, 0)
+    assert gh.max_excess(out, ref, wl.BF16) <= gh.TOL[wl.BF16]
+
+
 def test_prefill_output_aligned_to_16_bytes_only(prefill_kernel):
     """q and out start 16 bytes into their buffers: 16-byte aligned, not
     32.  The tcgen05 kernel then stores its rows in 16-byte pieces instead
