@@ -21,6 +21,19 @@ def test_decode_bytes_count_every_token_once():
     assert bench.algorithmic_bytes(lens, Hq, Hkv, d) == brute
 
 
+def test_append_bytes_add_the_new_rows_of_non_empty_sequences():
+    """pa_decode_append also reads each sequence's new K and V rows and writes
+    them into the cache; an empty sequence (L = 0) writes nothing."""
+    lens = np.array([0, 1, 16, 17, 1000], np.int64)
+    Hq, Hkv, d = 8, 2, 128
+    rows = 0
+    for L in lens:
+        if L > 0:
+            rows += 2 * Hkv * d * 2 * 2       # K and V rows: read k_new / v_new, write the cache
+    assert (bench.algorithmic_bytes(lens, Hq, Hkv, d, append=True)
+            == bench.algorithmic_bytes(lens, Hq, Hkv, d) + rows)
+
+
 def test_prefill_flops_match_a_per_query_count():
     lens = np.array([512, 700, 3000], np.int64)
     chunk, Hq, d = 512, 32, 128
