@@ -911,6 +911,7 @@ def run_cow_run(args, world, rank, local):
     ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=device)
     torch.cuda.synchronize(device)
     stream = torch.cuda.Stream(device)
+    fused = args.step == "fused"
 
     def run():
         for tables, lens, slots, pairs, n, _ in plan:
@@ -918,9 +919,13 @@ def run_cow_run(args, world, rank, local):
                 c = l % ncache
                 if pairs is not None:
                     pk.copy_blocks(kc[c], vc[c], pairs, stream=stream)
-                pk.reshape_and_cache(kn[l][:n], vn[l][:n], kc[c], vc[c], slots, stream=stream)
-                pk.decode(out[l][:n], q[l][:n], kc[c], vc[c], tables, lens, H, w.scale,
-                          workspace=ws, stream=stream)
+                if fused:
+                    pk.decode_append(out[l][:n], q[l][:n], kn[l][:n], vn[l][:n], kc[c], vc[c],
+                                     tables, lens, H, w.scale, workspace=ws, stream=stream)
+                else:
+                    pk.reshape_and_cache(kn[l][:n], vn[l][:n], kc[c], vc[c], slots, stream=stream)
+                    pk.decode(out[l][:n], q[l][:n], kc[c], vc[c], tables, lens, H, w.scale,
+                              workspace=ws, stream=stream)
 
     with torch.cuda.stream(stream):
         run()
@@ -968,9 +973,12 @@ def run_cow_run(args, world, rank, local):
                    "layer_caches": ncache, "timing": "whole run captured in one CUDA graph"},
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "traffic": None,
-                     "kernel": "whole run (copy + scatter + decode), logical bytes",
+                     "kernel": "whole run (copy + " + ("pa_decode_append" if fused else "scatter + decode")
+                               + "), logical bytes",
                      "peak_source": src},
-        "gpu_launches": args.steps * sum(L * (2 + (1 if p[3] is not None else 0) + 1)
+        "step": ("pa_copy_blocks (divergence step), " if any(p[3] is not None for p in plan) else "")
+                + ("pa_decode_append per layer" if fused else "pa_reshape_and_cache, pa_decode per layer"),
+        "gpu_launches": args.steps * sum(L * ((1 if fused else 2) + (1 if p[3] is not None else 0) + 1)
                                          for p in plan),
         "clocks": clocks}), flush=True)
 
