@@ -806,3 +806,65 @@ def test_a_wait_that_never_completes_times_out_and_the_context_survives():
     lens = np.array([600, 20], np.int32)
     p = make_paged(rng, 2, 8, 2, 128, lens, wl.blocks_needed(lens, 16), wl.BF16)
     assert gh.max_err(gpu_out(p), oracle_out(p)) <= gh.TOL[wl.BF16]
+
+
+# ---------------------------------------------------------------- seeded random configurations
+def random_config(seed):
+    """A seeded random problem: group size, head dim, dtype, kv heads, batch
+    size and context lengths (empty, short, block-aligned, multi-partition)."""
+    rng = wl.rng_for(900 + seed)
+    G = int(rng.choice([1, 2, 3, 4, 5, 8, 12, 16]))
+    hkv = int(rng.choice([1, 2, 4, 8]))
+    d = int(rng.choice([64, 128]))
+    dtype = wl.F16 if rng.random() < 0.5 else wl.BF16
+    S = int(rng.integers(1, 12))
+    kinds = rng.integers(0, 4, size=S)
+    lens = np.where(kinds == 0, rng.integers(0, 17, size=S),
+                    np.where(kinds == 1, 16 * rng.integers(1, 40, size=S),
+                             np.where(kinds == 2, rng.integers(17, 600, size=S),
+                                      rng.integers(600, 2500, size=S)))).astype(np.int32)
+    return rng, G * hkv, hkv, d, dtype, lens
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_configs_decode_append(seed):
+    """pa_decode_append and pa_reshape_and_cache + pa_decode on seeded random
+    configurations: equal to each other bit for bit, and to the oracle."""
+    rng, hq, hkv, d, dtype, lens = random_config(seed)
+    S = len(lens)
+    p = make_paged(rng, S, hq, hkv, d, lens, wl.blocks_needed(lens, 16) + 3, dtype)
+    k_new = wl.draw_values(rng, (S, hkv, d), dtype)
+    v_new = wl.draw_values(rng, (S, hkv, d), dtype)
+    slots = append_slots(p)
+    tbl, ln = gh.ints(p.tables), gh.ints(p.lens)
+    dk, dv, q = gh.to_dev(k_new, dtype), gh.to_dev(v_new, dtype), gh.to_dev(p.q, dtype)
+    ws = gh.workspace_for(pk, S, hq, d, p.tables.shape[1])
+    kc1, vc1 = gh.to_dev(p.key_cache, dtype), gh.to_dev(p.value_cache, dtype)
+    out1 = torch.full_like(q, float("nan"))
+    pk.reshape_and_cache(dk, dv, kc1, vc1, gh.ints(slots, torch.int64))
+    pk.decode(out1, q, kc1, vc1, tbl, ln, hkv, p.scale, workspace=ws)
+    kc2, vc2 = gh.to_dev(p.key_cache, dtype), gh.to_dev(p.value_cache, dtype)
+    out2 = torch.full_like(q, float("nan"))
+    pk.decode_append(out2, q, dk, dv, kc2, vc2, tbl, ln, hkv, p.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert pk.get_error() == (0, 0)
+    assert torch.equal(kc1, kc2) and torch.equal(vc1, vc2) and torch.equal(out1, out2)
+    oracle.reshape_and_cache(k_new, v_new, p.key_cache, p.value_cache, slots)
+    assert np.array_equal(gh.to_host_bits(kc2), p.key_cache)
+    assert gh.max_err(out2, oracle_out(p)) <= gh.TOL[dtype]
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_configs_prefill(seed, prefill_kernel):
+    """Chunked prefill on seeded random configurations (chunks from one token
+    to the whole context), on both kernels, against the oracle."""
+    rng, hq, hkv, d, dtype, lens = random_config(seed)
+    lens = np.maximum(lens, 1)
+    qlens = np.array([int(rng.integers(1, L + 1)) if rng.random() < 0.7 else int(L) for L in lens],
+                     np.int32)
+    qlens = np.minimum(qlens, 300).astype(np.int32)
+    p = make_paged(rng, len(lens), hq, hkv, d, lens, wl.blocks_needed(lens, 16) + 3, dtype)
+    qchunk = wl.draw_values(rng, (int(qlens.sum()), hq, d), dtype)
+    out, ref = run_prefill(p, qchunk, qlens)
+    assert pk.get_error() == (0, 0)
+    assert gh.max_excess(out, ref, dtype) <= gh.TOL[dtype]
