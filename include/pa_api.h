@@ -123,7 +123,8 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
  * "Continuous Batching Keeps the GPU Busy" (decode reads memory, not math).
  *
  * For sequence s with L = context_lens[s] cached tokens (the new token
- * included, written beforehand by pa_reshape_and_cache) and query head h,
+ * included, written beforehand by pa_reshape_and_cache; pa_decode_append
+ * does both in one launch) and query head h,
  * with G = num_q_heads / num_kv_heads and kv head g = h / G:
  *   K_j = key_cache  [block_tables[s][j / 16]][g][j % 16][:],  j < L
  *   V_j = value_cache[block_tables[s][j / 16]][g][j % 16][:]
