@@ -170,7 +170,9 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
  * followed by pa_decode(...) with the same arguments: the same cache bytes
  * afterwards, and the same outputs, bit for bit.  Sequences with L == 0
  * write nothing (zero output row).  An out-of-range block id at position
- * L - 1 writes nothing and sets PA_DEVERR_BLOCK_ID, as pa_decode reports it.
+ * L - 1 writes nothing and sets PA_DEVERR_BLOCK_ID, as pa_decode reports it;
+ * so does a context length beyond the table (PA_DEVERR_CONTEXT_LEN), whose
+ * position L - 1 has no slot.
  * The block holding position L - 1 must belong to this sequence alone (the
  * allocator copies a shared last block before appending to it): another
  * sequence that reads it in the same call may see the slot before or after

@@ -196,10 +196,12 @@ __device__ __forceinline__ int warp_block_count(int nb_local, int warp, int nw) 
 // this call (partitions are disjoint token ranges).
 //
 // append_block_index: the warp's own index k of that block (its k-th block
-// is b_begin + warp + k * nw), or -1 when another warp or CTA holds it.
-__device__ __forceinline__ int append_block_index(const DecodeArgs &a, int L, int b_begin,
+// is b_begin + warp + k * nw), or -1 when another warp or CTA holds it.  A
+// context length that had to be clamped to the table (reported as
+// PA_DEVERR_CONTEXT_LEN) writes nothing: position L - 1 is not in the table.
+__device__ __forceinline__ int append_block_index(const DecodeArgs &a, int s, int L, int b_begin,
                                                   int nb_local, int warp, int nw) {
-    if (a.k_new == nullptr || L <= 0) return -1;
+    if (a.k_new == nullptr || L <= 0 || a.context_lens[s] != L) return -1;
     const int li = (L - 1) / kBlock - b_begin;
     if (li < 0 || li >= nb_local || li % nw != warp) return -1;
     return li / nw;
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(NW * 32)
     // pa_decode_append: write the new token before the load of its block; if
     // that load is not among the first ones, after them, so that the write's
     // latency overlaps theirs
-    const int k_app = append_block_index(a, L, b_begin, nb_local, warp, NW);
+    const int k_app = append_block_index(a, s, L, b_begin, nb_local, warp, NW);
     if (k_app >= 0 && k_app < issued) append_new_token<D>(a, s, kvh, L, lane);
     for (int k = 0; k < issued; ++k) pipe.issue(k);
     if (k_app >= issued) append_new_token<D>(a, s, kvh, L, lane);
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? PA_DECODE_MIN_CTAS : 3)
     // pa_decode_append: write the new token before the load of its block; if
     // that load is not among the first ones, after them, so that the write's
     // latency overlaps theirs
-    const int k_app = append_block_index(a, L, b_begin, nb_local, warp, NW);
+    const int k_app = append_block_index(a, s, L, b_begin, nb_local, warp, NW);
     if (k_app >= 0 && k_app < issued) append_new_token<D>(a, s, kvh, L, lane);
     for (int k = 0; k < issued; ++k) pipe.issue(k);
     if (k_app >= issued) append_new_token<D>(a, s, kvh, L, lane);

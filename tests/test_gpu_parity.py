@@ -128,6 +128,36 @@ def test_decode_append_bad_last_block_writes_nothing():
     assert gh.max_err(out[[0, 2]], ref) <= gh.TOL[wl.BF16]
 
 
+def test_decode_append_context_beyond_the_table_writes_nothing():
+    """Sequence 1's context length runs past its table: reported as a bad
+    context length, its new row is written nowhere (the length is clamped
+    for the attention, but position L - 1 has no slot), the other sequence
+    is written and exact."""
+    rng = wl.rng_for(69)
+    lens = np.array([30, 32], np.int32)
+    p = make_paged(rng, 2, 4, 2, 64, lens, 6, wl.F16, max_blocks=2)
+    k_new = wl.draw_values(rng, (2, 2, 64), wl.F16)
+    v_new = wl.draw_values(rng, (2, 2, 64), wl.F16)
+    slots = append_slots(p)
+    bad = p.lens.copy()
+    bad[1] = 32 + 1000
+    kc, vc = gh.to_dev(p.key_cache, wl.F16), gh.to_dev(p.value_cache, wl.F16)
+    q = gh.to_dev(p.q, wl.F16)
+    out = torch.full_like(q, float("nan"))
+    pk.decode_append(out, q, gh.to_dev(k_new, wl.F16), gh.to_dev(v_new, wl.F16), kc, vc,
+                     gh.ints(p.tables), gh.ints(bad), 2, p.scale)
+    torch.cuda.synchronize()
+    rc, bits = pk.get_error()
+    assert rc == pk.PA_ERR_OUT_OF_RANGE and bits & pk.DEVERR_CONTEXT_LEN
+    slots[1] = -1
+    oracle.reshape_and_cache(k_new, v_new, p.key_cache, p.value_cache, slots)
+    assert np.array_equal(gh.to_host_bits(kc), p.key_cache)
+    assert np.array_equal(gh.to_host_bits(vc), p.value_cache)
+    ref = oracle.decode(p.q, p.key_cache, p.value_cache, p.tables, p.lens, 2, p.scale, wl.F16,
+                        seqs=[0])
+    assert gh.max_err(out[:1], ref) <= gh.TOL[wl.F16]
+
+
 def test_decode_append_checks_its_new_rows():
     rng = wl.rng_for(67)
     lens = np.array([5, 9], np.int32)
